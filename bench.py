@@ -1,0 +1,468 @@
+#!/usr/bin/env python
+"""Benchmark of the emulated RCCLX collectives on B200.
+
+One STEP is one pass of every hot-path operation over one batch of N=8
+simulated ranks x 16,777,216 fp32 elements (64 MiB per rank, N(0,1) with 1%
+of the elements scaled x100 as outliers -- the >= 16 MB low-precision message
+size the RCCLX pages target):
+
+    quantise, dequantise (128-block FP8 E4M3),
+    DDA-flat allreduce    (native fp32 wire, FP8 wire),
+    DDA-tree allreduce    (native fp32 wire, FP8 wire: fused
+                           dequantise-sum-requantise pass + all-gather pass),
+    reduce-scatter, all-gather, alltoall (native and FP8 wire).
+
+`value` is the effective HBM bandwidth of the whole step: the algorithmic
+bytes of all operations (inputs read once, outputs written once, plus the
+tree's wire payload written by pass 1 and read by pass 2) divided by the
+device time of the timed steps.  Every operation touches >= 576 MiB, far more
+than the 126 MB L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+With --gpus N > 1 (under torchrun) each GPU runs its own independent batch:
+there is no data-path exchange between GPUs (the emulated ranks all live in
+one GPU's memory), so the scaling is weak and `value` sums all GPUs.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+NRANKS = 8
+COUNT = 16_777_216
+M = COUNT // NRANKS
+BLOCK = 128
+MIB = 1 << 20
+WORKLOAD = 4        # seeded workload id in synth (N(0,1) + 1% x100 outliers)
+CPU_SAMPLE = 8_388_608   # elements per rank in the oracle's bounded sample (~10 s)
+
+
+# --------------------------------------------------------------- bytes model
+
+def op_bytes(count: int, nranks: int, esize: int = 4) -> dict[str, int]:
+    """Algorithmic HBM bytes per launch of each operation on [nranks][count]."""
+    n, c, m = nranks, count, count // nranks
+    nblk = (c + BLOCK - 1) // BLOCK
+    codes, scales = n * c, n * nblk * 4
+    data = n * c * esize
+    payload = c + nblk * 4                       # tree FP8 wire payload
+    return {
+        "quantize_fp8": data + codes + scales,
+        "dequantize_fp8": codes + scales + data,
+        "allreduce_flat_native": 2 * data,
+        "allreduce_flat_fp8": 2 * data,
+        "allreduce_tree_native": data + c * esize + c * esize + (n - 1) * c * esize,
+        "allreduce_tree_fp8": data + payload + payload + data,
+        "reduce_scatter_native": data + n * m * esize,
+        "reduce_scatter_fp8": data + n * m * esize,
+        "all_gather_native": n * m * esize + data,
+        "all_gather_fp8": n * m * esize + data,
+        "alltoall_native": 2 * data,
+        "alltoall_fp8": 2 * data,
+    }
+
+
+OPS = list(op_bytes(COUNT, NRANKS).keys())
+KERNELS_PER_OP = {op: (2 if op.startswith("allreduce_tree") else 1) for op in OPS}
+
+
+# ------------------------------------------------------------------ helpers
+
+def peaks() -> tuple[float, str]:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+def source_hash() -> str:
+    csrc = os.path.join(ROOT, "precision_collective_reduction_fp32_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(op: str):
+    """dram bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = rec.get(op)
+    if not e or e.get("src_sha") != source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples: list[tuple[float, int, int]] = []
+        self.period = period_s
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid).encode())
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001 -- clocks are reported as unavailable
+            self.err = repr(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self, t0: float, t1: float) -> dict:
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML: " + self.err}
+        self._stop.set()
+        self._t.join()
+        inside = [s for s in self.samples if t0 <= s[0] <= t1] or self.samples[-3:]
+        mhz = [s[1] for s in inside]
+        bits = 0
+        for s in inside:
+            bits |= s[2]
+        reasons = [name for b, name in self.REASONS.items() if bits & b and name != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(inside)}
+
+
+# ------------------------------------------------------------ the GPU step
+
+class Step:
+    """Device buffers for one batch and the twelve operations of one step,
+    each issued through the C ABI (librlx.so) on the current stream."""
+
+    def __init__(self, x_host: np.ndarray, device):
+        import torch
+        from precision_collective_reduction_fp32_b200 import binding as B
+        self.B, self.torch = B, torch
+        n, c = x_host.shape
+        self.n, self.c, self.m = n, c, c // n
+        t = lambda *s, dt=torch.float32: torch.empty(*s, dtype=dt, device=device)
+        self.x = torch.from_numpy(x_host).to(device)
+        self.out = t((n, c))
+        self.y = t((n, c))
+        self.codes = t((n, c), dt=torch.uint8)
+        self.scales = t((n, (c + BLOCK - 1) // BLOCK))
+        self.rs = t((n, self.m))
+        self.ws_bytes = B.rlx_workspace_bytes(B.RLX_COLL_ALLREDUCE_TREE, c, n, B.RLX_F32,
+                                              B.RLX_WIRE_FP8_E4M3)
+        self.ws = t((self.ws_bytes,), dt=torch.uint8)
+
+    def ops(self, stream):
+        B, n, c, m = self.B, self.n, self.c, self.m
+        x, out, y, rs = self.x.data_ptr(), self.out.data_ptr(), self.y.data_ptr(), self.rs.data_ptr()
+        F, NAT, FP8 = B.RLX_F32, B.RLX_WIRE_NATIVE, B.RLX_WIRE_FP8_E4M3
+        return [
+            ("quantize_fp8", lambda: B.rlx_quantize_fp8(x, F, n, c, c, self.codes.data_ptr(),
+                                                        self.scales.data_ptr(), stream)),
+            ("dequantize_fp8", lambda: B.rlx_dequantize_fp8(self.codes.data_ptr(), self.scales.data_ptr(),
+                                                            n, c, c, y, F, stream)),
+            ("allreduce_flat_native", lambda: B.rlx_allreduce_flat(x, out, c, c, n, F, NAT, B.RLX_SUM, stream)),
+            ("allreduce_flat_fp8", lambda: B.rlx_allreduce_flat(x, out, c, c, n, F, FP8, B.RLX_SUM, stream)),
+            ("allreduce_tree_native", lambda: B.rlx_allreduce_tree(x, out, c, c, n, F, NAT, B.RLX_SUM,
+                                                                   None, 0, stream)),
+            ("allreduce_tree_fp8", lambda: B.rlx_allreduce_tree(x, out, c, c, n, F, FP8, B.RLX_SUM,
+                                                                self.ws.data_ptr(), self.ws_bytes, stream)),
+            ("reduce_scatter_native", lambda: B.rlx_reduce_scatter(x, c, rs, m, m, n, F, NAT, B.RLX_SUM, stream)),
+            ("reduce_scatter_fp8", lambda: B.rlx_reduce_scatter(x, c, rs, m, m, n, F, FP8, B.RLX_SUM, stream)),
+            ("all_gather_native", lambda: B.rlx_all_gather(rs, m, y, c, m, n, F, NAT, stream)),
+            ("all_gather_fp8", lambda: B.rlx_all_gather(rs, m, y, c, m, n, F, FP8, stream)),
+            ("alltoall_native", lambda: B.rlx_alltoall(x, c, y, c, m, n, F, NAT, stream)),
+            ("alltoall_fp8", lambda: B.rlx_alltoall(x, c, y, c, m, n, F, FP8, stream)),
+        ]
+
+
+def run_gpu(args, rank: int, world: int) -> dict | None:
+    import torch
+    import torch.distributed as dist
+    from precision_collective_reduction_fp32_b200 import synth
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    # each GPU gets its own independent batch (different seeds per GPU)
+    count = args.count
+    x_host = np.empty((NRANKS, count), dtype=np.float32)
+    for r in range(NRANKS):
+        x_host[r] = synth.draw_row("normal_outliers", count, synth.seed(WORKLOAD, r) + 100 * rank)
+    step = Step(x_host, dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream or None
+    ops = step.ops(sp)
+    if args.only:
+        ops = [(n, f) for n, f in ops if n in args.only.split(",")]
+        assert ops, "unknown --only operation"
+    bytes_ = {n: b for n, b in op_bytes(count, NRANKS).items() if n in dict(ops)}
+    step_bytes = sum(bytes_.values())
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        for _, f in ops:
+            f()
+    torch.cuda.synchronize()
+
+    # ---- device-timed region: K steps, an event between every operation
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(ops) + 1)] for _ in range(K)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for k in range(K):
+        ev[k][0].record(stream)
+        for i, (_, f) in enumerate(ops):
+            f()
+            ev[k][i + 1].record(stream)
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    barrier()
+    clk = clocks.stop(t0, t1)
+    per_op_ms = {name: 0.0 for name, _ in ops}
+    for k in range(K):
+        for i, (name, _) in enumerate(ops):
+            per_op_ms[name] += ev[k][i].elapsed_time(ev[k][i + 1])
+    total_ms = ev[0][0].elapsed_time(ev[K - 1][-1])
+    t_dev = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_dev, op=dist.ReduceOp.MAX)
+    total_ms = float(t_dev.item())
+
+    # ---- end to end: pinned host -> device, the step, result -> host
+    host_in = torch.from_numpy(x_host).pin_memory()
+    host_out = torch.empty((NRANKS, count), dtype=torch.float32).pin_memory()
+    Ke = max(1, min(K, args.e2e_steps))
+    for _ in range(2):
+        step.x.copy_(host_in, non_blocking=True)
+        for _, f in ops:
+            f()
+        host_out.copy_(step.out, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(Ke):
+        step.x.copy_(host_in, non_blocking=True)
+        for _, f in ops:
+            f()
+        host_out.copy_(step.out, non_blocking=True)   # the FP8 tree allreduce result
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_dev = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e_dev, op=dist.ReduceOp.MAX)
+    e2e_ms = float(e_dev.item())
+    barrier()
+    if rank != 0:
+        return None
+
+    peak, peak_kind = peaks()
+    value = world * step_bytes * K / (total_ms * 1e-3) / 1e9
+    per_op = {}
+    for name in per_op_ms:
+        ms = per_op_ms[name] / K
+        gbs = bytes_[name] / (ms * 1e-3) / 1e9
+        per_op[name] = {"us": round(ms * 1e3, 2), "GB/s": round(gbs, 1),
+                        "frac": round(gbs / peak, 3), "MiB": round(bytes_[name] / MIB, 1)}
+    single = [n for n in per_op_ms if KERNELS_PER_OP[n] == 1]
+    dom = max(single, key=lambda n: per_op_ms[n])
+    dom_gbs = per_op[dom]["GB/s"]
+    traffic = recorded_traffic(dom)
+    res = {
+        "metric": "emulated N=8 allreduce effective HBM GB/s (fp32 & FP8) and % of B200 HBM peak",
+        "value": round(value, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / K, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": {
+            "workload": "N=8 simulated ranks x fp32[16,777,216] (64 MiB/rank), N(0,1) with 1% "
+                        "x100 outliers; one step = quantise, dequantise, DDA-flat and DDA-tree "
+                        "allreduce (native and FP8 wire), reduce-scatter, all-gather, alltoall "
+                        "(native and FP8 wire)",
+            "nranks": NRANKS, "count": count, "elem": "fp32", "fp8": "e4m3, 128-block fp32 scales",
+            "bytes_per_step": step_bytes,
+            "l2": "no flush: every operation streams >= 576 MiB, > 126 MB L2",
+            "parallelism": "independent batch per GPU" if world > 1 else "single GPU",
+        },
+        "hbm_frac": round(value / world / peak, 3),
+        "ops": per_op,
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": dom_gbs, "peak": peak,
+                     "unit": "GB/s", "frac": round(dom_gbs / peak, 3), "traffic": traffic,
+                     "algorithmic_bytes": bytes_[dom], "peak_kind": peak_kind},
+        "gpu_launches": K * sum(KERNELS_PER_OP[n] for n in bytes_),
+        "clocks": clk,
+        "e2e": {"value": round(world * step_bytes * Ke / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                "h2d_bytes_per_step": NRANKS * count * 4, "d2h_bytes_per_step": NRANKS * count * 4,
+                "ms_per_step": round(e2e_ms / Ke, 3), "steps": Ke},
+    }
+    if count != COUNT or args.only:
+        res["config"]["workload"] = "PROFILING CASE, not the benchmark: %s on N=8 x fp32[%d]" % (
+            ",".join(bytes_), count)
+    if world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(x_host, sample=min(CPU_SAMPLE, count))
+    return res
+
+
+# --------------------------------------------------------------- CPU oracle
+
+def oracle_step(xs: np.ndarray) -> None:
+    """The same twelve operations, run by the CPU oracle on a sample."""
+    import oracle
+    n, c = xs.shape
+    m = c // n
+    codes, scales = oracle.quantize(xs)
+    oracle.dequantize(codes, scales)
+    for w in (oracle.NATIVE, oracle.FP8):
+        oracle.allreduce_flat(xs, wire=w)
+        oracle.allreduce_tree(xs, wire=w)
+        rs = oracle.reduce_scatter(xs, m, wire=w)
+        oracle.all_gather(rs, m, wire=w)
+        oracle.alltoall(xs, m, wire=w)
+
+
+def cpu_baseline(x_host: np.ndarray, sample: int = CPU_SAMPLE, repeats: int = 1) -> dict:
+    import oracle
+    oracle.build()
+    xs = np.ascontiguousarray(x_host[:, :sample])
+    t0 = time.perf_counter()
+    for _ in range(repeats):
+        oracle_step(xs)
+    dt = time.perf_counter() - t0
+    b = sum(op_bytes(sample, NRANKS).values()) * repeats
+    return {"value": round(b / dt / 1e9, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "host_cores": os.cpu_count(),
+            "sample": "%d pass(es) of the twelve operations on the first %d elements of each of "
+                      "the %d ranks (1/%d of the batch), single-threaded C oracle; %.1f s"
+                      % (repeats, sample, NRANKS, COUNT // sample, dt)}
+
+
+def run_reference(args, rank: int) -> dict | None:
+    """The reference arm: the CPU oracle as it stands, on bounded samples."""
+    if rank != 0:
+        return None
+    from precision_collective_reduction_fp32_b200 import synth
+    sample = args.ref_sample
+    xs = np.empty((NRANKS, sample), dtype=np.float32)
+    for r in range(NRANKS):
+        xs[r] = synth.draw_row("normal_outliers", sample, synth.seed(WORKLOAD, r))
+    for _ in range(args.warmup):
+        oracle_step(xs)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(xs)
+    dt = time.perf_counter() - t0
+    b = sum(op_bytes(sample, NRANKS).values()) * args.steps
+    value = b / dt / 1e9
+    desc = ("each step: the twelve operations on the first %d elements of each of the %d ranks "
+            "(1/%d of the batch), single-threaded C oracle" % (sample, NRANKS, COUNT // sample))
+    return {"impl": "reference",
+            "metric": "emulated N=8 allreduce effective HBM GB/s (fp32 & FP8) and % of B200 HBM peak",
+            "value": round(value, 3), "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": "N=8 simulated ranks x fp32[16,777,216], N(0,1) with 1% x100 "
+                                   "outliers (bounded sample, see cpu_baseline)",
+                       "nranks": NRANKS, "count": COUNT},
+            "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": 1,
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["rlx", "reference"], default="rlx")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--ref-sample", type=int, default=262_144)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--count", type=int, default=COUNT,
+                    help="elements per rank (profiling cases only; the benchmark is 16,777,216)")
+    ap.add_argument("--only", default="",
+                    help="comma-separated operations to run (profiling cases only)")
+    args = ap.parse_args(argv)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        res = run_gpu(args, rank, world)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if res is not None:
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

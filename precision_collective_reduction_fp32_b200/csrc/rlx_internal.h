@@ -1,0 +1,63 @@
+// rlx_internal.h -- launcher interface between the C ABI layer (rlx_api.cu)
+// and the kernel translation units.  Arguments reaching these functions have
+// already been validated; `vec` says the vectorised kernels may be used
+// (every row and chunk start is aligned as the kernel requires).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/rlx.h"
+
+namespace rlx {
+
+constexpr int kThreads = 256;  // threads per CTA for every kernel
+
+// Grid for a persistent kernel: enough CTAs for `jobs` units of work at
+// `jobs_per_cta` each, capped at (resident CTAs per SM) x (SM count).
+int persistent_grid(const void *kernel, size_t jobs, size_t jobs_per_cta);
+
+// DDA-flat, all wires.  nranks >= 2.
+cudaError_t launch_allreduce_flat(const void *send, void *recv, size_t count, size_t stride,
+                                  int nranks, rlx_dtype dtype, rlx_wire wire, bool vec,
+                                  cudaStream_t stream);
+
+// DDA-tree pass 1 (reduce-scatter).  Native: writes chunk c into recv row c.
+// FP8: writes the requantised chunk codes/scales into the workspace.
+cudaError_t launch_tree_reduce(const void *send, void *recv, size_t count, size_t stride,
+                               int nranks, size_t chunk, rlx_dtype dtype, rlx_wire wire,
+                               uint8_t *ws_codes, float *ws_scales, bool vec,
+                               cudaStream_t stream);
+
+// DDA-tree pass 2 (all-gather).
+cudaError_t launch_tree_gather(void *recv, size_t count, size_t stride, int nranks,
+                               size_t chunk, rlx_dtype dtype, rlx_wire wire,
+                               const uint8_t *ws_codes, const float *ws_scales, bool vec,
+                               cudaStream_t stream);
+
+cudaError_t launch_reduce_scatter(const void *send, size_t send_stride, void *recv,
+                                  size_t recv_stride, size_t m, int nranks, rlx_dtype dtype,
+                                  rlx_wire wire, bool vec, cudaStream_t stream);
+
+cudaError_t launch_all_gather(const void *send, size_t send_stride, void *recv,
+                              size_t recv_stride, size_t m, int nranks, rlx_dtype dtype,
+                              rlx_wire wire, bool vec, cudaStream_t stream);
+
+cudaError_t launch_alltoall(const void *send, size_t send_stride, void *recv,
+                            size_t recv_stride, size_t m, int nranks, rlx_dtype dtype,
+                            rlx_wire wire, bool vec, cudaStream_t stream);
+
+// Row copy (every collective with one rank): dst[j] = src[j], j < n.
+cudaError_t launch_copy(const void *src, void *dst, size_t n, rlx_dtype dtype, bool vec,
+                        cudaStream_t stream);
+
+cudaError_t launch_quantize(const void *x, rlx_dtype dtype, size_t rows, size_t n,
+                            size_t stride, uint8_t *codes, float *scales, bool vec,
+                            cudaStream_t stream);
+
+cudaError_t launch_dequantize(const uint8_t *codes, const float *scales, size_t rows,
+                              size_t n, size_t stride, void *y, rlx_dtype dtype, bool vec,
+                              cudaStream_t stream);
+
+}  // namespace rlx

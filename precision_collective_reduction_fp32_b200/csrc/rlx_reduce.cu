@@ -1,0 +1,312 @@
+// rlx_reduce.cu -- the reducing passes: DDA-flat allreduce, DDA-tree pass 1
+// (reduce-scatter into chunk owners) and the standalone ReduceScatter, each on
+// the native wire and on the FP8 wire.
+//
+// DDA-flat: every rank reads every rank's buffer and reduces locally
+// ("Meta open-sources RCCLX", infolabhq pt, "Direct Data Access (DDA) — De
+// O(N) para O(1) de Latência").  On one GPU the N identical local reductions
+// are one reduction per element index whose result is stored into all N rows.
+// DDA-tree pass 1: rank c reduces chunk c (same section).  LP collectives:
+// each sender's contribution is quantised to FP8 and dequantised by the
+// receiver, sums are FP32 (RCCLX post, es, "Colectivos de mengua precisión").
+//
+// Work mapping
+//   native wire: one thread per 16-byte vector of each row (4 fp32 or 8 bf16);
+//     the thread loads that vector from all N ranks before adding, so N
+//     16-byte loads are in flight per thread;
+//   FP8 wire: one warp per 128-element block, 4 elements per lane, so the
+//     block amax is one warp reduction; the warp loads the block from all N
+//     ranks, dequantises each rank's quantised block, sums in rank order.
+// Grids are persistent (grid-stride loops) and sized from the occupancy.
+#include "rlx_device.cuh"
+#include "rlx_internal.h"
+
+namespace rlx {
+namespace {
+
+// ------------------------------------------------------ native 16-byte vectors
+
+template <typename T> struct VecN { static constexpr int n = 16 / sizeof(T); };
+
+// V consecutive elements as fp32; `valid` of them real, the rest +0.
+template <typename T, bool VEC>
+__device__ __forceinline__ void loadv(const T *p, int valid, float (&v)[VecN<T>::n]) {
+    constexpr int V = VecN<T>::n;
+    if (VEC && valid == V) {
+        const uint4 q = __ldcs(reinterpret_cast<const uint4 *>(p));
+        if constexpr (sizeof(T) == 4) {
+            v[0] = __uint_as_float(q.x); v[1] = __uint_as_float(q.y);
+            v[2] = __uint_as_float(q.z); v[3] = __uint_as_float(q.w);
+        } else {
+            const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                v[2 * k] = __uint_as_float(w[k] << 16);
+                v[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < V; ++k) v[k] = k < valid ? Elem<T>::load(p + k) : 0.0f;
+    }
+}
+
+template <typename T, bool VEC>
+__device__ __forceinline__ void storev(T *p, int valid, const float (&v)[VecN<T>::n]) {
+    constexpr int V = VecN<T>::n;
+    if (VEC && valid == V) {
+        uint4 q;
+        if constexpr (sizeof(T) == 4) {
+            q.x = __float_as_uint(v[0]); q.y = __float_as_uint(v[1]);
+            q.z = __float_as_uint(v[2]); q.w = __float_as_uint(v[3]);
+        } else {
+            uint32_t w[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                w[k] = static_cast<uint32_t>(f32_to_bf16_bits(v[2 * k])) |
+                       (static_cast<uint32_t>(f32_to_bf16_bits(v[2 * k + 1])) << 16);
+            q = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        __stcs(reinterpret_cast<uint4 *>(p), q);
+    } else {
+#pragma unroll
+        for (int k = 0; k < V; ++k)
+            if (k < valid) Elem<T>::store(p + k, v[k]);
+    }
+}
+
+// acc = x_0 + x_1 + ... + x_{n-1} (rank order) of the vector at `src` in each
+// of the n rows (row pitch `pitch` elements).  All loads are issued first.
+template <typename T, int NR, bool VEC>
+__device__ __forceinline__ void reduce_vec(const T *src, size_t pitch, int n, int valid,
+                                           float (&acc)[VecN<T>::n]) {
+    constexpr int V = VecN<T>::n;
+    float x[NR][V];
+#pragma unroll
+    for (int s = 0; s < NR; ++s)
+        if (s < n) loadv<T, VEC>(src + s * pitch, valid, x[s]);
+#pragma unroll
+    for (int k = 0; k < V; ++k) acc[k] = x[0][k];
+#pragma unroll
+    for (int s = 1; s < NR; ++s)
+        if (s < n) {
+#pragma unroll
+            for (int k = 0; k < V; ++k) acc[k] = __fadd_rn(acc[k], x[s][k]);
+        }
+}
+
+// ---------------------------------------------------- FP8 wire, warp per block
+
+// acc = SUM_s wire(x_s) over the 128-block at `src` in each of n rows, 4
+// elements per lane.  Lanes past the block end hold +0.
+template <typename T, int NR, bool VEC>
+__device__ __forceinline__ void reduce_block_fp8(const T *src, size_t pitch, int n, int valid,
+                                                 float (&acc)[4]) {
+    float x[NR][4];
+    const int e0 = lane_id() * 4;
+#pragma unroll
+    for (int s = 0; s < NR; ++s)
+        if (s < n) load4<T, VEC>(src + s * pitch + e0, valid, x[s]);
+    wire_fp8_block(x[0]);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc[k] = x[0][k];
+#pragma unroll
+    for (int s = 1; s < NR; ++s)
+        if (s < n) {
+            wire_fp8_block(x[s]);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[k] = __fadd_rn(acc[k], x[s][k]);
+        }
+}
+
+// ------------------------------------------------------------------ kernels
+
+template <typename T, int NR, bool VEC>
+__global__ void __launch_bounds__(kThreads)
+flat_native_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
+    constexpr int V = VecN<T>::n;
+    const size_t nvec = (count + V - 1) / V;
+    const size_t step = static_cast<size_t>(gridDim.x) * blockDim.x;
+    for (size_t v = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < nvec; v += step) {
+        const size_t i0 = v * V;
+        const int valid = count - i0 < static_cast<size_t>(V) ? static_cast<int>(count - i0) : V;
+        float acc[V];
+        reduce_vec<T, NR, VEC>(send + i0, stride, n, valid, acc);
+        for (int r = 0; r < n; ++r) storev<T, VEC>(recv + r * stride + i0, valid, acc);
+    }
+}
+
+template <typename T, int NR, bool VEC>
+__global__ void __launch_bounds__(kThreads)
+flat_fp8_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
+    const size_t nblk = (count + kBlock - 1) / kBlock;
+    const int e0 = lane_id() * 4;
+    for (size_t b = global_warp(); b < nblk; b += num_warps()) {
+        const size_t base = b * kBlock;
+        const int len = count - base < static_cast<size_t>(kBlock) ? static_cast<int>(count - base) : kBlock;
+        const int valid = lane_valid(len);
+        float acc[4];
+        reduce_block_fp8<T, NR, VEC>(send + base, stride, n, valid, acc);
+        for (int r = 0; r < n; ++r) store4<T, VEC>(recv + r * stride + base + e0, valid, acc);
+    }
+}
+
+// DDA-tree pass 1, native: chunk c -> row c of recv.
+template <typename T, int NR, bool VEC>
+__global__ void __launch_bounds__(kThreads)
+tree_reduce_native_kernel(const T *send, T *recv, size_t count, size_t stride, int n,
+                          size_t chunk) {
+    constexpr int V = VecN<T>::n;
+    const size_t step = static_cast<size_t>(gridDim.x) * blockDim.x;
+    const size_t tid = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    for (int c = 0; c < n; ++c) {
+        const size_t lo = static_cast<size_t>(c) * chunk;
+        if (lo >= count) break;
+        const size_t hi = count - lo < chunk ? count : lo + chunk;
+        const size_t nvec = (hi - lo + V - 1) / V;
+        for (size_t v = tid; v < nvec; v += step) {
+            const size_t i0 = lo + v * V;
+            const int valid = hi - i0 < static_cast<size_t>(V) ? static_cast<int>(hi - i0) : V;
+            float acc[V];
+            reduce_vec<T, NR, VEC>(send + i0, stride, n, valid, acc);
+            storev<T, VEC>(recv + c * stride + i0, valid, acc);
+        }
+    }
+}
+
+// DDA-tree pass 1, FP8: reduce, then quantise the reduced block again into
+// the workspace payload (codes padded to whole blocks, one scale per block).
+template <typename T, int NR, bool VEC>
+__global__ void __launch_bounds__(kThreads)
+tree_reduce_fp8_kernel(const T *send, size_t count, size_t stride, int n,
+                       uint8_t *ws_codes, float *ws_scales) {
+    const size_t nblk = (count + kBlock - 1) / kBlock;
+    const int e0 = lane_id() * 4;
+    for (size_t b = global_warp(); b < nblk; b += num_warps()) {
+        const size_t base = b * kBlock;
+        const int len = count - base < static_cast<size_t>(kBlock) ? static_cast<int>(count - base) : kBlock;
+        float acc[4];
+        reduce_block_fp8<T, NR, VEC>(send + base, stride, n, lane_valid(len), acc);
+        const float s = block_scale(warp_amax4(acc));
+        const uint32_t codes = quant4(acc, s);
+        // default caching: the payload is read back by pass 2 right away
+        *reinterpret_cast<uint32_t *>(ws_codes + base + e0) = codes;
+        if (lane_id() == 0) ws_scales[b] = s;
+    }
+}
+
+template <typename T, int NR, bool VEC>
+__global__ void __launch_bounds__(kThreads)
+rs_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n) {
+    constexpr int V = VecN<T>::n;
+    const size_t step = static_cast<size_t>(gridDim.x) * blockDim.x;
+    const size_t tid = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const size_t nvec = (m + V - 1) / V;
+    for (int r = 0; r < n; ++r) {
+        for (size_t v = tid; v < nvec; v += step) {
+            const size_t j0 = v * V;
+            const int valid = m - j0 < static_cast<size_t>(V) ? static_cast<int>(m - j0) : V;
+            float acc[V];
+            reduce_vec<T, NR, VEC>(send + r * m + j0, sstride, n, valid, acc);
+            storev<T, VEC>(recv + r * rstride + j0, valid, acc);
+        }
+    }
+}
+
+template <typename T, int NR, bool VEC>
+__global__ void __launch_bounds__(kThreads)
+rs_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n) {
+    const size_t nbm = (m + kBlock - 1) / kBlock;
+    const size_t jobs = nbm * static_cast<size_t>(n);
+    const int e0 = lane_id() * 4;
+    for (size_t job = global_warp(); job < jobs; job += num_warps()) {
+        const size_t r = job / nbm;
+        const size_t j0 = (job - r * nbm) * kBlock;
+        const int len = m - j0 < static_cast<size_t>(kBlock) ? static_cast<int>(m - j0) : kBlock;
+        const int valid = lane_valid(len);
+        float acc[4];
+        reduce_block_fp8<T, NR, VEC>(send + r * m + j0, sstride, n, valid, acc);
+        store4<T, VEC>(recv + r * rstride + j0 + e0, valid, acc);
+    }
+}
+
+// ------------------------------------------------------------- dispatching
+
+// Calls f.template operator()<T, NR, VEC>() for the rank bound NR >= n.
+template <typename F>
+cudaError_t dispatch(rlx_dtype dtype, int n, bool vec, F &&f) {
+#define RLX_CASE_NR(T, NRV)                                                       \
+    if (n <= NRV) return vec ? f.template operator()<T, NRV, true>()              \
+                             : f.template operator()<T, NRV, false>();
+#define RLX_CASE_T(T) \
+    RLX_CASE_NR(T, 2) RLX_CASE_NR(T, 4) RLX_CASE_NR(T, 8) RLX_CASE_NR(T, 16)
+    if (dtype == RLX_F32) { RLX_CASE_T(float) }
+    else { RLX_CASE_T(uint16_t) }
+#undef RLX_CASE_T
+#undef RLX_CASE_NR
+    return cudaErrorInvalidValue;
+}
+
+template <typename K, typename... Args>
+cudaError_t launch(K kernel, size_t jobs, size_t jobs_per_cta, cudaStream_t stream, Args... args) {
+    const int grid = persistent_grid(reinterpret_cast<const void *>(kernel), jobs, jobs_per_cta);
+    kernel<<<grid, kThreads, 0, stream>>>(args...);
+    return cudaGetLastError();
+}
+
+constexpr size_t kWarps = kThreads / 32;
+
+}  // namespace
+
+cudaError_t launch_allreduce_flat(const void *send, void *recv, size_t count, size_t stride,
+                                  int nranks, rlx_dtype dtype, rlx_wire wire, bool vec,
+                                  cudaStream_t stream) {
+    return dispatch(dtype, nranks, vec, [&]<typename T, int NR, bool VEC>() {
+        const T *s = static_cast<const T *>(send);
+        T *r = static_cast<T *>(recv);
+        if (wire == RLX_WIRE_NATIVE) {
+            const size_t nvec = (count + VecN<T>::n - 1) / VecN<T>::n;
+            return launch(flat_native_kernel<T, NR, VEC>, nvec, kThreads, stream, s, r, count,
+                          stride, nranks);
+        }
+        const size_t nblk = (count + kBlock - 1) / kBlock;
+        return launch(flat_fp8_kernel<T, NR, VEC>, nblk, kWarps, stream, s, r, count, stride,
+                      nranks);
+    });
+}
+
+cudaError_t launch_tree_reduce(const void *send, void *recv, size_t count, size_t stride,
+                               int nranks, size_t chunk, rlx_dtype dtype, rlx_wire wire,
+                               uint8_t *ws_codes, float *ws_scales, bool vec,
+                               cudaStream_t stream) {
+    return dispatch(dtype, nranks, vec, [&]<typename T, int NR, bool VEC>() {
+        const T *s = static_cast<const T *>(send);
+        if (wire == RLX_WIRE_NATIVE) {
+            const size_t nvec = (chunk + VecN<T>::n - 1) / VecN<T>::n;
+            return launch(tree_reduce_native_kernel<T, NR, VEC>, nvec, kThreads, stream, s,
+                          static_cast<T *>(recv), count, stride, nranks, chunk);
+        }
+        const size_t nblk = (count + kBlock - 1) / kBlock;
+        return launch(tree_reduce_fp8_kernel<T, NR, VEC>, nblk, kWarps, stream, s, count,
+                      stride, nranks, ws_codes, ws_scales);
+    });
+}
+
+cudaError_t launch_reduce_scatter(const void *send, size_t send_stride, void *recv,
+                                  size_t recv_stride, size_t m, int nranks, rlx_dtype dtype,
+                                  rlx_wire wire, bool vec, cudaStream_t stream) {
+    return dispatch(dtype, nranks, vec, [&]<typename T, int NR, bool VEC>() {
+        const T *s = static_cast<const T *>(send);
+        T *r = static_cast<T *>(recv);
+        if (wire == RLX_WIRE_NATIVE) {
+            const size_t nvec = (m + VecN<T>::n - 1) / VecN<T>::n;
+            return launch(rs_native_kernel<T, NR, VEC>, nvec, kThreads, stream, s, send_stride,
+                          r, recv_stride, m, nranks);
+        }
+        const size_t jobs = (m + kBlock - 1) / kBlock * static_cast<size_t>(nranks);
+        return launch(rs_fp8_kernel<T, NR, VEC>, jobs, kWarps, stream, s, send_stride, r,
+                      recv_stride, m, nranks);
+    });
+}
+
+}  // namespace rlx
