@@ -11,7 +11,8 @@
 
 namespace rlx {
 
-int persistent_grid(const void *kernel, size_t jobs, size_t jobs_per_cta) {
+dim3 grid_2d(const void *kernel, unsigned segments, size_t jobs_per_segment,
+             size_t jobs_per_cta) {
     static std::mutex mu;
     static std::map<std::pair<int, const void *>, int> cap_cache;
     int dev = 0;
@@ -31,9 +32,13 @@ int persistent_grid(const void *kernel, size_t jobs, size_t jobs_per_cta) {
             cap_cache[{dev, kernel}] = cap;
         }
     }
-    const size_t need = (jobs + jobs_per_cta - 1) / jobs_per_cta;
-    if (need == 0) return 1;
-    return need < static_cast<size_t>(cap) ? static_cast<int>(need) : cap;
+    if (segments == 0) segments = 1;
+    size_t need = (jobs_per_segment + jobs_per_cta - 1) / jobs_per_cta;
+    if (need == 0) need = 1;
+    size_t share = (static_cast<size_t>(cap) + segments - 1) / segments;
+    if (share == 0) share = 1;
+    const size_t x = need < share ? need : share;
+    return dim3(static_cast<unsigned>(x), segments, 1);
 }
 
 }  // namespace rlx

@@ -1,11 +1,11 @@
 // rlx_device.cuh -- device-side building blocks shared by the rlx kernels.
 //
-// Element access (vectorised 16/8-byte or element-wise), the FP8 E4M3 codec on
-// the hardware cvt instructions, the warp-wide block amax, and the "wire"
-// transform dequantise(quantise(x)) of one 128-element block held as 4 values
-// per lane of a warp.  Every floating-point step is an explicit
+// Element access (vectorised or element-wise), the FP8 E4M3 codec on the
+// hardware cvt instructions, the warp-wide block amax, the block scale and the
+// "wire" transform dequantise(quantise(x)) of 128-element blocks held as 4
+// values per lane of a warp.  Every floating-point step is an explicit
 // round-to-nearest intrinsic so that the compiler cannot contract a multiply
-// and an add into an FMA.
+// and an add into an FMA that the definition does not have.
 #pragma once
 
 #include <cstddef>
@@ -19,6 +19,10 @@ namespace rlx {
 constexpr int kBlock = 128;        // elements per FP8 scale block
 constexpr float kE4m3Max = 448.0f; // largest finite E4M3 magnitude
 constexpr unsigned kFull = 0xffffffffu;
+// Below this block scale the quotient x/s falls back to the IEEE division
+// (see quotient_rn); at or above it every residual that can change a code is
+// exact.  2^-90.
+constexpr float kMinFastScale = 0x1p-90f;
 
 // ------------------------------------------------------------ element types
 
@@ -30,15 +34,13 @@ __device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
     return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
 
-// Element traits: load/store one element as fp32.
+// Element traits: load/store one element as fp32 (streaming cache hints).
 template <typename T> struct Elem;
 template <> struct Elem<float> {
-    using storage = float;
     __device__ __forceinline__ static float load(const float *p) { return __ldcs(p); }
     __device__ __forceinline__ static void store(float *p, float v) { __stcs(p, v); }
 };
 template <> struct Elem<uint16_t> {  // bf16 bit patterns
-    using storage = uint16_t;
     __device__ __forceinline__ static float load(const uint16_t *p) {
         return bf16_bits_to_f32(__ldcs(reinterpret_cast<const unsigned short *>(p)));
     }
@@ -53,10 +55,10 @@ template <typename T, bool VEC>
 __device__ __forceinline__ void load4(const T *p, int valid, float (&v)[4]) {
     if (VEC && valid == 4) {
         if constexpr (sizeof(T) == 4) {
-            float4 q = __ldcs(reinterpret_cast<const float4 *>(p));
+            const float4 q = __ldcs(reinterpret_cast<const float4 *>(p));
             v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
         } else {
-            uint2 q = __ldcs(reinterpret_cast<const uint2 *>(p));
+            const uint2 q = __ldcs(reinterpret_cast<const uint2 *>(p));
             v[0] = __uint_as_float(q.x << 16);
             v[1] = __uint_as_float(q.x & 0xffff0000u);
             v[2] = __uint_as_float(q.y << 16);
@@ -114,32 +116,80 @@ __device__ __forceinline__ float2 e4m3x2_to_f32(uint32_t two_codes) {
     return __half22float2(__half2(raw));  // every E4M3 value is exact in f16 and f32
 }
 
-// ------------------------------------------------------------ block helpers
+// ------------------------------------------------------------ block scales
 
-// max |v| over the 4 values of every lane of the warp (all 32 lanes must call).
+// max |v| over the 4 values of every lane of the warp (all 32 lanes call).
 // For non-negative floats the IEEE bit order is the value order, so the warp
 // reduction runs on the integer bits.
 __device__ __forceinline__ float warp_amax4(const float (&v)[4]) {
-    uint32_t m = __float_as_uint(v[0]) & 0x7fffffffu;
-    m = max(m, __float_as_uint(v[1]) & 0x7fffffffu);
-    m = max(m, __float_as_uint(v[2]) & 0x7fffffffu);
-    m = max(m, __float_as_uint(v[3]) & 0x7fffffffu);
-    return __uint_as_float(__reduce_max_sync(kFull, m));
+    const float m = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+    return __uint_as_float(__reduce_max_sync(kFull, __float_as_uint(m)));
 }
 
-// Block scale s = fl32(amax / 448), correctly rounded.
-__device__ __forceinline__ float block_scale(float amax) { return __fdiv_rn(amax, kE4m3Max); }
+// Scale of a block: s = fl32(amax / 448), and y = fl32(1 / s) when the fast
+// quotient may be used (s >= 2^-90), else 0.
+struct Scale {
+    float s, y;
+};
+__device__ __forceinline__ Scale make_scale(float amax) {
+    Scale r;
+    r.s = __fdiv_rn(amax, kE4m3Max);
+    r.y = r.s >= kMinFastScale ? __frcp_rn(r.s) : 0.0f;
+    return r;
+}
 
-// Quantise 4 values with scale s: code = e4m3_rne_sat(fl32(v / s)); s == 0
-// gives signed zeros.
-__device__ __forceinline__ uint32_t quant4(const float (&v)[4], float s) {
+// Scales of K blocks held by the warp at once (K <= 32, a power of two).
+// Lane l computes the division and the reciprocal for block l % K only; the
+// results are then broadcast, so a lane pays for one division instead of K.
+template <int K>
+__device__ __forceinline__ void make_scales(const float (&amax)[K], Scale (&sc)[K]) {
+    static_assert(K >= 1 && K <= 32 && (K & (K - 1)) == 0, "K must be a power of two <= 32");
+    const int mine = threadIdx.x & (K - 1);
+    float a = amax[0];
+#pragma unroll
+    for (int k = 1; k < K; ++k)
+        if (mine == k) a = amax[k];
+    const Scale m = make_scale(a);
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+        sc[k].s = __shfl_sync(kFull, m.s, k);
+        sc[k].y = __shfl_sync(kFull, m.y, k);
+    }
+}
+
+// fl32(x / s), correctly rounded, from y = fl32(1/s) (s >= 2^-90).
+// Markstein's division theorem (P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1),
+// 1990): if y approximates 1/s with relative error below 2^-24 and q is a
+// faithful approximation of x/s, then r = x - s*q is exact and q + r*y
+// rounded to nearest is the correctly rounded quotient.  q0 = x*y can be up to
+// 1.5 ulp away, so one correction first makes it faithful, the second rounds
+// it correctly.  With s >= 2^-90 every residual that can affect an E4M3 code
+// (|x/s| >= 2^-10) is exact; smaller quotients only need their sign and a
+// magnitude below 2^-10, which the steps keep.  The sign is copied from x so
+// that x = -0 gives -0.
+__device__ __forceinline__ float quotient_rn(float x, float s, float y) {
+    float q = __fmul_rn(x, y);
+    float r = __fmaf_rn(-s, q, x);
+    q = __fmaf_rn(r, y, q);
+    r = __fmaf_rn(-s, q, x);
+    q = __fmaf_rn(r, y, q);
+    return copysignf(q, x);
+}
+
+// Quantise 4 values of a block with scale sc: code = e4m3_rne_sat(fl32(v/s));
+// s == 0 gives signed zeros.  sc.y == 0 selects the IEEE division.
+__device__ __forceinline__ uint32_t quant4(const float (&v)[4], Scale sc) {
     float q[4];
-    if (s == 0.0f) {
+    if (sc.y != 0.0f) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) q[k] = quotient_rn(v[k], sc.s, sc.y);
+    } else if (sc.s == 0.0f) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) q[k] = __fmul_rn(v[k], 0.0f);  // +-0 with v's sign
     } else {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) q[k] = __fdiv_rn(v[k], s);
+        for (int k = 0; k < 4; ++k) q[k] = __fdiv_rn(v[k], sc.s);
     }
     return e4m3x4_from_f32(q);
 }
@@ -154,27 +204,42 @@ __device__ __forceinline__ void dequant4(uint32_t codes, float s, float (&y)[4])
     y[3] = __fmul_rn(b.y, s);
 }
 
-// What a receiver holds after one 128-block crossed the FP8 wire: the warp
-// holds the block as 4 values per lane (lanes past the end hold +0, which
-// leaves amax unchanged); returns dequantise(quantise(v)) in place.
-__device__ __forceinline__ void wire_fp8_block(float (&v)[4]) {
-    const float s = block_scale(warp_amax4(v));
-    dequant4(quant4(v, s), s, v);
+// What a receiver holds after K 128-blocks crossed the FP8 wire.  The warp
+// holds block k as 4 values per lane in v[k] (lanes past a block's end hold
+// +0, which leaves its amax unchanged).  In place.
+template <int K>
+__device__ __forceinline__ void wire_fp8_blocks(float (&v)[K][4]) {
+    float amax[K];
+#pragma unroll
+    for (int k = 0; k < K; ++k) amax[k] = warp_amax4(v[k]);
+    Scale sc[K];
+    make_scales<K>(amax, sc);
+#pragma unroll
+    for (int k = 0; k < K; ++k) dequant4(quant4(v[k], sc[k]), sc[k].s, v[k]);
 }
 
 // ----------------------------------------------------------- grid helpers
 
-__device__ __forceinline__ size_t global_warp() {
+__device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
+__device__ __forceinline__ size_t warp_in_grid_x() {
     return (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
 }
-__device__ __forceinline__ size_t num_warps() {
+__device__ __forceinline__ size_t warps_in_grid_x() {
     return (static_cast<size_t>(gridDim.x) * blockDim.x) >> 5;
 }
-__device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
+__device__ __forceinline__ size_t thread_in_grid_x() {
+    return static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+}
+__device__ __forceinline__ size_t threads_in_grid_x() {
+    return static_cast<size_t>(gridDim.x) * blockDim.x;
+}
 
 // Elements of a 128-block that belong to this lane: 0..4.
-__device__ __forceinline__ int lane_valid(int block_len) {
-    const int v = block_len - lane_id() * 4;
+__device__ __forceinline__ int lane_valid(size_t block_start, size_t len) {
+    if (block_start >= len) return 0;
+    const size_t rem = len - block_start;
+    const int blen = rem < static_cast<size_t>(kBlock) ? static_cast<int>(rem) : kBlock;
+    const int v = blen - lane_id() * 4;
     return v < 0 ? 0 : (v > 4 ? 4 : v);
 }
 

@@ -9,37 +9,63 @@
 // quantises what it sends and the receiver dequantises it.
 //
 // On the native wire these passes move bytes only (16-byte vectors, no
-// conversion), so results are bit copies.  On the FP8 wire one warp handles
-// one 128-element block (4 elements per lane): it reads the block once,
-// applies dequantise(quantise(.)) in registers and writes every destination.
+// conversion), so results are bit copies; each thread keeps kUnroll vectors in
+// flight.  On the FP8 wire a warp handles kJ consecutive 128-element blocks
+// at once (4 elements per lane per block): it reads them, applies
+// dequantise(quantise(.)) in registers and writes every destination.
+// Per-chunk work uses a 2-D grid (y = source rank, rank pair or chunk).
 #include "rlx_device.cuh"
 #include "rlx_internal.h"
 
 namespace rlx {
 namespace {
 
-// Copy V = 16/sizeof(T) elements (valid of them) as raw bits.
+constexpr int kUnroll = 4;  // 16-byte vectors in flight per thread (native copies)
+constexpr int kJ = 4;       // 128-blocks in flight per warp (FP8 single-source)
+constexpr int kJd = 8;      // 128-blocks per warp when reading FP8 payloads
+
+template <typename T> constexpr int kV = 16 / sizeof(T);
+
+// One 16-byte vector (valid elements of it) as raw bits.
 template <typename T, bool VEC>
-__device__ __forceinline__ void copyv_load(const T *p, int valid, uint4 &q, T (&e)[16 / sizeof(T)]) {
-    constexpr int V = 16 / sizeof(T);
-    if (VEC && valid == V) {
-        q = __ldcs(reinterpret_cast<const uint4 *>(p));
-    } else {
+struct RawVec {
+    uint4 q;
+    T e[kV<T>];
+    __device__ __forceinline__ void load(const T *p, int valid) {
+        if (VEC && valid == kV<T>) {
+            q = __ldcs(reinterpret_cast<const uint4 *>(p));
+        } else {
 #pragma unroll
-        for (int k = 0; k < V; ++k)
-            if (k < valid) e[k] = p[k];
+            for (int k = 0; k < kV<T>; ++k)
+                if (k < valid) e[k] = p[k];
+        }
     }
-}
-template <typename T, bool VEC>
-__device__ __forceinline__ void copyv_store(T *p, int valid, const uint4 &q, const T (&e)[16 / sizeof(T)]) {
-    constexpr int V = 16 / sizeof(T);
-    if (VEC && valid == V) {
-        __stcs(reinterpret_cast<uint4 *>(p), q);
-    } else {
+    // default caching, for data written by the previous pass
+    __device__ __forceinline__ void load_cached(const T *p, int valid) {
+        if (VEC && valid == kV<T>) {
+            q = *reinterpret_cast<const uint4 *>(p);
+        } else {
 #pragma unroll
-        for (int k = 0; k < V; ++k)
-            if (k < valid) p[k] = e[k];
+            for (int k = 0; k < kV<T>; ++k)
+                if (k < valid) e[k] = p[k];
+        }
     }
+    __device__ __forceinline__ void store(T *p, int valid) const {
+        if (VEC && valid == kV<T>) {
+            __stcs(reinterpret_cast<uint4 *>(p), q);
+        } else {
+#pragma unroll
+            for (int k = 0; k < kV<T>; ++k)
+                if (k < valid) p[k] = e[k];
+        }
+    }
+};
+
+template <typename T>
+__device__ __forceinline__ int vec_valid(size_t v, size_t nvec, size_t len) {
+    if (v >= nvec) return 0;
+    const size_t rem = len - v * kV<T>;
+    return rem < static_cast<size_t>(kV<T>) ? static_cast<int>(rem) : kV<T>;
 }
 
 // ------------------------------------------------------------------ kernels
@@ -47,141 +73,171 @@ __device__ __forceinline__ void copyv_store(T *p, int valid, const uint4 &q, con
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 copy_kernel(const T *src, T *dst, size_t n) {
-    constexpr int V = 16 / sizeof(T);
-    const size_t nvec = (n + V - 1) / V;
-    const size_t step = static_cast<size_t>(gridDim.x) * blockDim.x;
-    for (size_t v = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < nvec; v += step) {
-        const size_t i0 = v * V;
-        const int valid = n - i0 < static_cast<size_t>(V) ? static_cast<int>(n - i0) : V;
-        uint4 q;
-        T e[V];
-        copyv_load<T, VEC>(src + i0, valid, q, e);
-        copyv_store<T, VEC>(dst + i0, valid, q, e);
+    const size_t nvec = (n + kV<T> - 1) / kV<T>;
+    const size_t T_ = threads_in_grid_x();
+    for (size_t v0 = thread_in_grid_x(); v0 < nvec; v0 += kUnroll * T_) {
+        RawVec<T, VEC> a[kUnroll];
+        int valid[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            valid[u] = vec_valid<T>(v0 + u * T_, nvec, n);
+            if (valid[u]) a[u].load(src + (v0 + u * T_) * kV<T>, valid[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u)
+            if (valid[u]) a[u].store(dst + (v0 + u * T_) * kV<T>, valid[u]);
     }
 }
 
-// DDA-tree pass 2, native: chunk c of row c -> chunk c of every other row.
+// DDA-tree pass 2, native: chunk c = blockIdx.y of row c -> every other row.
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 tree_gather_native_kernel(T *recv, size_t count, size_t stride, int n, size_t chunk) {
-    constexpr int V = 16 / sizeof(T);
-    const size_t step = static_cast<size_t>(gridDim.x) * blockDim.x;
-    const size_t tid = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    for (int c = 0; c < n; ++c) {
-        const size_t lo = static_cast<size_t>(c) * chunk;
-        if (lo >= count) break;
-        const size_t hi = count - lo < chunk ? count : lo + chunk;
-        const size_t nvec = (hi - lo + V - 1) / V;
-        for (size_t v = tid; v < nvec; v += step) {
-            const size_t i0 = lo + v * V;
-            const int valid = hi - i0 < static_cast<size_t>(V) ? static_cast<int>(hi - i0) : V;
-            uint4 q;
-            T e[V];
-            // the owner's chunk was just written by pass 1: default caching
-            if (VEC && valid == V) q = *reinterpret_cast<const uint4 *>(recv + c * stride + i0);
-            else copyv_load<T, false>(recv + c * stride + i0, valid, q, e);
-            for (int r = 0; r < n; ++r)
-                if (r != c) copyv_store<T, VEC>(recv + r * stride + i0, valid, q, e);
+    const int c = blockIdx.y;
+    const size_t lo = static_cast<size_t>(c) * chunk;
+    if (lo >= count) return;
+    const size_t len = count - lo < chunk ? count - lo : chunk;
+    const size_t nvec = (len + kV<T> - 1) / kV<T>;
+    const size_t T_ = threads_in_grid_x();
+    const T *src = recv + c * stride + lo;
+    for (size_t v0 = thread_in_grid_x(); v0 < nvec; v0 += kUnroll * T_) {
+        RawVec<T, VEC> a[kUnroll];
+        int valid[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            valid[u] = vec_valid<T>(v0 + u * T_, nvec, len);
+            if (valid[u]) a[u].load_cached(src + (v0 + u * T_) * kV<T>, valid[u]);
+        }
+        for (int r = 0; r < n; ++r) {
+            if (r == c) continue;
+            T *dst = recv + r * stride + lo;
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u)
+                if (valid[u]) a[u].store(dst + (v0 + u * T_) * kV<T>, valid[u]);
         }
     }
 }
 
-// DDA-tree pass 2, FP8: dequantise the payload block into every row.
+// DDA-tree pass 2, FP8: dequantise the payload blocks into every row.
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 tree_gather_fp8_kernel(T *recv, size_t count, size_t stride, int n, const uint8_t *ws_codes,
                        const float *ws_scales) {
     const size_t nblk = (count + kBlock - 1) / kBlock;
     const int e0 = lane_id() * 4;
-    for (size_t b = global_warp(); b < nblk; b += num_warps()) {
-        const size_t base = b * kBlock;
-        const int len = count - base < static_cast<size_t>(kBlock) ? static_cast<int>(count - base) : kBlock;
-        const int valid = lane_valid(len);
-        const uint32_t codes = *reinterpret_cast<const uint32_t *>(ws_codes + base + e0);
-        const float s = ws_scales[b];
-        float y[4];
-        dequant4(codes, s, y);
-        for (int r = 0; r < n; ++r) store4<T, VEC>(recv + r * stride + base + e0, valid, y);
+    for (size_t b0 = warp_in_grid_x() * kJd; b0 < nblk; b0 += warps_in_grid_x() * kJd) {
+        float y[kJd][4];
+        int valid[kJd];
+#pragma unroll
+        for (int j = 0; j < kJd; ++j) {
+            const size_t b = b0 + j;
+            valid[j] = lane_valid(b * kBlock, count);
+            if (b < nblk) {
+                const uint32_t codes = *reinterpret_cast<const uint32_t *>(ws_codes + b * kBlock + e0);
+                dequant4(codes, ws_scales[b], y[j]);
+            }
+        }
+        for (int r = 0; r < n; ++r)
+#pragma unroll
+            for (int j = 0; j < kJd; ++j)
+                store4<T, VEC>(recv + r * stride + (b0 + j) * kBlock + e0, valid[j], y[j]);
     }
 }
 
+// AllGather, native: source rank s = blockIdx.y.
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 ag_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n) {
-    constexpr int V = 16 / sizeof(T);
-    const size_t step = static_cast<size_t>(gridDim.x) * blockDim.x;
-    const size_t tid = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    const size_t nvec = (m + V - 1) / V;
-    for (int s = 0; s < n; ++s) {
-        for (size_t v = tid; v < nvec; v += step) {
-            const size_t j0 = v * V;
-            const int valid = m - j0 < static_cast<size_t>(V) ? static_cast<int>(m - j0) : V;
-            uint4 q;
-            T e[V];
-            copyv_load<T, VEC>(send + s * sstride + j0, valid, q, e);
-            for (int r = 0; r < n; ++r) copyv_store<T, VEC>(recv + r * rstride + s * m + j0, valid, q, e);
+    const size_t s = blockIdx.y;
+    const size_t nvec = (m + kV<T> - 1) / kV<T>;
+    const size_t T_ = threads_in_grid_x();
+    const T *src = send + s * sstride;
+    for (size_t v0 = thread_in_grid_x(); v0 < nvec; v0 += kUnroll * T_) {
+        RawVec<T, VEC> a[kUnroll];
+        int valid[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            valid[u] = vec_valid<T>(v0 + u * T_, nvec, m);
+            if (valid[u]) a[u].load(src + (v0 + u * T_) * kV<T>, valid[u]);
+        }
+        for (int r = 0; r < n; ++r) {
+            T *dst = recv + r * rstride + s * m;
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u)
+                if (valid[u]) a[u].store(dst + (v0 + u * T_) * kV<T>, valid[u]);
         }
     }
 }
 
+// AllGather, FP8: source rank s = blockIdx.y; blocks anchored at its row start.
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 ag_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n) {
+    const size_t s = blockIdx.y;
     const size_t nbm = (m + kBlock - 1) / kBlock;
-    const size_t jobs = nbm * static_cast<size_t>(n);
     const int e0 = lane_id() * 4;
-    for (size_t job = global_warp(); job < jobs; job += num_warps()) {
-        const size_t s = job / nbm;
-        const size_t j0 = (job - s * nbm) * kBlock;
-        const int len = m - j0 < static_cast<size_t>(kBlock) ? static_cast<int>(m - j0) : kBlock;
-        const int valid = lane_valid(len);
-        float v[4];
-        load4<T, VEC>(send + s * sstride + j0 + e0, valid, v);
-        wire_fp8_block(v);
-        for (int r = 0; r < n; ++r) store4<T, VEC>(recv + r * rstride + s * m + j0 + e0, valid, v);
-    }
-}
-
-template <typename T, bool VEC>
-__global__ void __launch_bounds__(kThreads)
-a2a_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n) {
-    constexpr int V = 16 / sizeof(T);
-    const size_t step = static_cast<size_t>(gridDim.x) * blockDim.x;
-    const size_t tid = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    const size_t nvec = (m + V - 1) / V;
-    for (int s = 0; s < n; ++s) {
+    const T *src = send + s * sstride;
+    for (size_t b0 = warp_in_grid_x() * kJ; b0 < nbm; b0 += warps_in_grid_x() * kJ) {
+        float v[kJ][4];
+        int valid[kJ];
+#pragma unroll
+        for (int j = 0; j < kJ; ++j) {
+            valid[j] = lane_valid((b0 + j) * kBlock, m);
+            load4<T, VEC>(src + (b0 + j) * kBlock + e0, valid[j], v[j]);
+        }
+        wire_fp8_blocks<kJ>(v);
         for (int r = 0; r < n; ++r) {
-            const T *src = send + s * sstride + r * m;
             T *dst = recv + r * rstride + s * m;
-            for (size_t v = tid; v < nvec; v += step) {
-                const size_t j0 = v * V;
-                const int valid = m - j0 < static_cast<size_t>(V) ? static_cast<int>(m - j0) : V;
-                uint4 q;
-                T e[V];
-                copyv_load<T, VEC>(src + j0, valid, q, e);
-                copyv_store<T, VEC>(dst + j0, valid, q, e);
-            }
+#pragma unroll
+            for (int j = 0; j < kJ; ++j) store4<T, VEC>(dst + (b0 + j) * kBlock + e0, valid[j], v[j]);
         }
     }
 }
 
+// AlltoAll, native: pair = blockIdx.y = s * n + r moves chunk r of rank s to
+// chunk s of rank r.
+template <typename T, bool VEC>
+__global__ void __launch_bounds__(kThreads)
+a2a_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n) {
+    const size_t s = blockIdx.y / n, r = blockIdx.y % n;
+    const T *src = send + s * sstride + r * m;
+    T *dst = recv + r * rstride + s * m;
+    const size_t nvec = (m + kV<T> - 1) / kV<T>;
+    const size_t T_ = threads_in_grid_x();
+    for (size_t v0 = thread_in_grid_x(); v0 < nvec; v0 += kUnroll * T_) {
+        RawVec<T, VEC> a[kUnroll];
+        int valid[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            valid[u] = vec_valid<T>(v0 + u * T_, nvec, m);
+            if (valid[u]) a[u].load(src + (v0 + u * T_) * kV<T>, valid[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u)
+            if (valid[u]) a[u].store(dst + (v0 + u * T_) * kV<T>, valid[u]);
+    }
+}
+
+// AlltoAll, FP8: pair = blockIdx.y; blocks anchored at the chunk start r*m.
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 a2a_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n) {
+    const size_t s = blockIdx.y / n, r = blockIdx.y % n;
+    const T *src = send + s * sstride + r * m;
+    T *dst = recv + r * rstride + s * m;
     const size_t nbm = (m + kBlock - 1) / kBlock;
-    const size_t nn = static_cast<size_t>(n);
-    const size_t jobs = nbm * nn * nn;
     const int e0 = lane_id() * 4;
-    for (size_t job = global_warp(); job < jobs; job += num_warps()) {
-        const size_t pair = job / nbm;          // pair = s * n + r
-        const size_t j0 = (job - pair * nbm) * kBlock;
-        const size_t s = pair / nn, r = pair - s * nn;
-        const int len = m - j0 < static_cast<size_t>(kBlock) ? static_cast<int>(m - j0) : kBlock;
-        const int valid = lane_valid(len);
-        float v[4];
-        load4<T, VEC>(send + s * sstride + r * m + j0 + e0, valid, v);
-        wire_fp8_block(v);
-        store4<T, VEC>(recv + r * rstride + s * m + j0 + e0, valid, v);
+    for (size_t b0 = warp_in_grid_x() * kJ; b0 < nbm; b0 += warps_in_grid_x() * kJ) {
+        float v[kJ][4];
+        int valid[kJ];
+#pragma unroll
+        for (int j = 0; j < kJ; ++j) {
+            valid[j] = lane_valid((b0 + j) * kBlock, m);
+            load4<T, VEC>(src + (b0 + j) * kBlock + e0, valid[j], v[j]);
+        }
+        wire_fp8_blocks<kJ>(v);
+#pragma unroll
+        for (int j = 0; j < kJ; ++j) store4<T, VEC>(dst + (b0 + j) * kBlock + e0, valid[j], v[j]);
     }
 }
 
@@ -195,22 +251,26 @@ cudaError_t dispatch(rlx_dtype dtype, bool vec, F &&f) {
 }
 
 template <typename K, typename... Args>
-cudaError_t launch(K kernel, size_t jobs, size_t jobs_per_cta, cudaStream_t stream, Args... args) {
-    const int grid = persistent_grid(reinterpret_cast<const void *>(kernel), jobs, jobs_per_cta);
+cudaError_t launch(K kernel, unsigned segments, size_t jobs_per_segment, size_t jobs_per_cta,
+                   cudaStream_t stream, Args... args) {
+    const dim3 grid = grid_2d(reinterpret_cast<const void *>(kernel), segments,
+                              jobs_per_segment, jobs_per_cta);
     kernel<<<grid, kThreads, 0, stream>>>(args...);
     return cudaGetLastError();
 }
 
 constexpr size_t kWarps = kThreads / 32;
 
+template <typename T> size_t nvec_of(size_t n) { return (n + kV<T> - 1) / kV<T>; }
+size_t nblk_of(size_t n) { return (n + kBlock - 1) / kBlock; }
+
 }  // namespace
 
 cudaError_t launch_copy(const void *src, void *dst, size_t n, rlx_dtype dtype, bool vec,
                         cudaStream_t stream) {
     return dispatch(dtype, vec, [&]<typename T, bool VEC>() {
-        const size_t nvec = (n + 16 / sizeof(T) - 1) / (16 / sizeof(T));
-        return launch(copy_kernel<T, VEC>, nvec, kThreads, stream, static_cast<const T *>(src),
-                      static_cast<T *>(dst), n);
+        return launch(copy_kernel<T, VEC>, 1, nvec_of<T>(n), kThreads * kUnroll, stream,
+                      static_cast<const T *>(src), static_cast<T *>(dst), n);
     });
 }
 
@@ -220,14 +280,12 @@ cudaError_t launch_tree_gather(void *recv, size_t count, size_t stride, int nran
                                cudaStream_t stream) {
     return dispatch(dtype, vec, [&]<typename T, bool VEC>() {
         T *r = static_cast<T *>(recv);
-        if (wire == RLX_WIRE_NATIVE) {
-            const size_t nvec = (chunk + 16 / sizeof(T) - 1) / (16 / sizeof(T));
-            return launch(tree_gather_native_kernel<T, VEC>, nvec, kThreads, stream, r, count,
-                          stride, nranks, chunk);
-        }
-        const size_t nblk = (count + kBlock - 1) / kBlock;
-        return launch(tree_gather_fp8_kernel<T, VEC>, nblk, kWarps, stream, r, count, stride,
-                      nranks, ws_codes, ws_scales);
+        if (wire == RLX_WIRE_NATIVE)
+            return launch(tree_gather_native_kernel<T, VEC>, static_cast<unsigned>(nranks),
+                          nvec_of<T>(chunk), kThreads * kUnroll, stream, r, count, stride,
+                          nranks, chunk);
+        return launch(tree_gather_fp8_kernel<T, VEC>, 1, nblk_of(count), kWarps * kJd, stream, r,
+                      count, stride, nranks, ws_codes, ws_scales);
     });
 }
 
@@ -237,14 +295,12 @@ cudaError_t launch_all_gather(const void *send, size_t send_stride, void *recv,
     return dispatch(dtype, vec, [&]<typename T, bool VEC>() {
         const T *s = static_cast<const T *>(send);
         T *r = static_cast<T *>(recv);
-        if (wire == RLX_WIRE_NATIVE) {
-            const size_t nvec = (m + 16 / sizeof(T) - 1) / (16 / sizeof(T));
-            return launch(ag_native_kernel<T, VEC>, nvec, kThreads, stream, s, send_stride, r,
-                          recv_stride, m, nranks);
-        }
-        const size_t jobs = (m + kBlock - 1) / kBlock * static_cast<size_t>(nranks);
-        return launch(ag_fp8_kernel<T, VEC>, jobs, kWarps, stream, s, send_stride, r,
-                      recv_stride, m, nranks);
+        const unsigned segs = static_cast<unsigned>(nranks);
+        if (wire == RLX_WIRE_NATIVE)
+            return launch(ag_native_kernel<T, VEC>, segs, nvec_of<T>(m), kThreads * kUnroll, stream,
+                          s, send_stride, r, recv_stride, m, nranks);
+        return launch(ag_fp8_kernel<T, VEC>, segs, nblk_of(m), kWarps * kJ, stream, s,
+                      send_stride, r, recv_stride, m, nranks);
     });
 }
 
@@ -254,15 +310,12 @@ cudaError_t launch_alltoall(const void *send, size_t send_stride, void *recv,
     return dispatch(dtype, vec, [&]<typename T, bool VEC>() {
         const T *s = static_cast<const T *>(send);
         T *r = static_cast<T *>(recv);
-        if (wire == RLX_WIRE_NATIVE) {
-            const size_t nvec = (m + 16 / sizeof(T) - 1) / (16 / sizeof(T));
-            return launch(a2a_native_kernel<T, VEC>, nvec, kThreads, stream, s, send_stride, r,
-                          recv_stride, m, nranks);
-        }
-        const size_t nn = static_cast<size_t>(nranks);
-        const size_t jobs = (m + kBlock - 1) / kBlock * nn * nn;
-        return launch(a2a_fp8_kernel<T, VEC>, jobs, kWarps, stream, s, send_stride, r,
-                      recv_stride, m, nranks);
+        const unsigned pairs = static_cast<unsigned>(nranks * nranks);
+        if (wire == RLX_WIRE_NATIVE)
+            return launch(a2a_native_kernel<T, VEC>, pairs, nvec_of<T>(m), kThreads * kUnroll,
+                          stream, s, send_stride, r, recv_stride, m, nranks);
+        return launch(a2a_fp8_kernel<T, VEC>, pairs, nblk_of(m), kWarps * kJ, stream, s,
+                      send_stride, r, recv_stride, m, nranks);
     });
 }
 

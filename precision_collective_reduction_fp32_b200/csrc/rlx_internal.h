@@ -14,9 +14,12 @@ namespace rlx {
 
 constexpr int kThreads = 256;  // threads per CTA for every kernel
 
-// Grid for a persistent kernel: enough CTAs for `jobs` units of work at
-// `jobs_per_cta` each, capped at (resident CTAs per SM) x (SM count).
-int persistent_grid(const void *kernel, size_t jobs, size_t jobs_per_cta);
+// Grid for a persistent kernel over `segments` equal segments of work (grid
+// y) of `jobs_per_segment` units each, `jobs_per_cta` units per CTA and loop
+// iteration: x = enough CTAs for one segment, capped so that all segments
+// together use about (resident CTAs per SM) x (SM count) CTAs.
+dim3 grid_2d(const void *kernel, unsigned segments, size_t jobs_per_segment,
+             size_t jobs_per_cta);
 
 // DDA-flat, all wires.  nranks >= 2.
 cudaError_t launch_allreduce_flat(const void *send, void *recv, size_t count, size_t stride,

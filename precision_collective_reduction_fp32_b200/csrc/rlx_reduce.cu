@@ -14,10 +14,11 @@
 //   native wire: one thread per 16-byte vector of each row (4 fp32 or 8 bf16);
 //     the thread loads that vector from all N ranks before adding, so N
 //     16-byte loads are in flight per thread;
-//   FP8 wire: one warp per 128-element block, 4 elements per lane, so the
-//     block amax is one warp reduction; the warp loads the block from all N
-//     ranks, dequantises each rank's quantised block, sums in rank order.
-// Grids are persistent (grid-stride loops) and sized from the occupancy.
+//   FP8 wire: one warp per 128-element block, 4 elements per lane, so a block
+//     amax is one warp reduction; the warp loads the block from all N ranks,
+//     dequantises each rank's quantised block and sums in rank order.
+// Chunked passes use a 2-D grid (y = chunk / destination rank), so no thread
+// divides indices and every chunk gets the same share of the grid.
 #include "rlx_device.cuh"
 #include "rlx_internal.h"
 
@@ -98,22 +99,27 @@ __device__ __forceinline__ void reduce_vec(const T *src, size_t pitch, int n, in
 // ---------------------------------------------------- FP8 wire, warp per block
 
 // acc = SUM_s wire(x_s) over the 128-block at `src` in each of n rows, 4
-// elements per lane.  Lanes past the block end hold +0.
+// elements per lane (`valid` of them real; the rest +0).
 template <typename T, int NR, bool VEC>
 __device__ __forceinline__ void reduce_block_fp8(const T *src, size_t pitch, int n, int valid,
                                                  float (&acc)[4]) {
     float x[NR][4];
     const int e0 = lane_id() * 4;
 #pragma unroll
-    for (int s = 0; s < NR; ++s)
-        if (s < n) load4<T, VEC>(src + s * pitch + e0, valid, x[s]);
-    wire_fp8_block(x[0]);
+    for (int s = 0; s < NR; ++s) {
+        if (s < n) {
+            load4<T, VEC>(src + s * pitch + e0, valid, x[s]);
+        } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) x[s][k] = 0.0f;
+        }
+    }
+    wire_fp8_blocks<NR>(x);
 #pragma unroll
     for (int k = 0; k < 4; ++k) acc[k] = x[0][k];
 #pragma unroll
     for (int s = 1; s < NR; ++s)
         if (s < n) {
-            wire_fp8_block(x[s]);
 #pragma unroll
             for (int k = 0; k < 4; ++k) acc[k] = __fadd_rn(acc[k], x[s][k]);
         }
@@ -126,8 +132,7 @@ __global__ void __launch_bounds__(kThreads)
 flat_native_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
     constexpr int V = VecN<T>::n;
     const size_t nvec = (count + V - 1) / V;
-    const size_t step = static_cast<size_t>(gridDim.x) * blockDim.x;
-    for (size_t v = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < nvec; v += step) {
+    for (size_t v = thread_in_grid_x(); v < nvec; v += threads_in_grid_x()) {
         const size_t i0 = v * V;
         const int valid = count - i0 < static_cast<size_t>(V) ? static_cast<int>(count - i0) : V;
         float acc[V];
@@ -141,36 +146,32 @@ __global__ void __launch_bounds__(kThreads)
 flat_fp8_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
     const size_t nblk = (count + kBlock - 1) / kBlock;
     const int e0 = lane_id() * 4;
-    for (size_t b = global_warp(); b < nblk; b += num_warps()) {
+    for (size_t b = warp_in_grid_x(); b < nblk; b += warps_in_grid_x()) {
         const size_t base = b * kBlock;
-        const int len = count - base < static_cast<size_t>(kBlock) ? static_cast<int>(count - base) : kBlock;
-        const int valid = lane_valid(len);
+        const int valid = lane_valid(base, count);
         float acc[4];
         reduce_block_fp8<T, NR, VEC>(send + base, stride, n, valid, acc);
         for (int r = 0; r < n; ++r) store4<T, VEC>(recv + r * stride + base + e0, valid, acc);
     }
 }
 
-// DDA-tree pass 1, native: chunk c -> row c of recv.
+// DDA-tree pass 1, native: chunk c = blockIdx.y -> row c of recv.
 template <typename T, int NR, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 tree_reduce_native_kernel(const T *send, T *recv, size_t count, size_t stride, int n,
                           size_t chunk) {
     constexpr int V = VecN<T>::n;
-    const size_t step = static_cast<size_t>(gridDim.x) * blockDim.x;
-    const size_t tid = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    for (int c = 0; c < n; ++c) {
-        const size_t lo = static_cast<size_t>(c) * chunk;
-        if (lo >= count) break;
-        const size_t hi = count - lo < chunk ? count : lo + chunk;
-        const size_t nvec = (hi - lo + V - 1) / V;
-        for (size_t v = tid; v < nvec; v += step) {
-            const size_t i0 = lo + v * V;
-            const int valid = hi - i0 < static_cast<size_t>(V) ? static_cast<int>(hi - i0) : V;
-            float acc[V];
-            reduce_vec<T, NR, VEC>(send + i0, stride, n, valid, acc);
-            storev<T, VEC>(recv + c * stride + i0, valid, acc);
-        }
+    const int c = blockIdx.y;
+    const size_t lo = static_cast<size_t>(c) * chunk;
+    if (lo >= count) return;
+    const size_t hi = count - lo < chunk ? count : lo + chunk;
+    const size_t nvec = (hi - lo + V - 1) / V;
+    for (size_t v = thread_in_grid_x(); v < nvec; v += threads_in_grid_x()) {
+        const size_t i0 = lo + v * V;
+        const int valid = hi - i0 < static_cast<size_t>(V) ? static_cast<int>(hi - i0) : V;
+        float acc[V];
+        reduce_vec<T, NR, VEC>(send + i0, stride, n, valid, acc);
+        storev<T, VEC>(recv + c * stride + i0, valid, acc);
     }
 }
 
@@ -182,48 +183,45 @@ tree_reduce_fp8_kernel(const T *send, size_t count, size_t stride, int n,
                        uint8_t *ws_codes, float *ws_scales) {
     const size_t nblk = (count + kBlock - 1) / kBlock;
     const int e0 = lane_id() * 4;
-    for (size_t b = global_warp(); b < nblk; b += num_warps()) {
+    for (size_t b = warp_in_grid_x(); b < nblk; b += warps_in_grid_x()) {
         const size_t base = b * kBlock;
-        const int len = count - base < static_cast<size_t>(kBlock) ? static_cast<int>(count - base) : kBlock;
         float acc[4];
-        reduce_block_fp8<T, NR, VEC>(send + base, stride, n, lane_valid(len), acc);
-        const float s = block_scale(warp_amax4(acc));
-        const uint32_t codes = quant4(acc, s);
-        // default caching: the payload is read back by pass 2 right away
+        reduce_block_fp8<T, NR, VEC>(send + base, stride, n, lane_valid(base, count), acc);
+        const Scale sc = make_scale(warp_amax4(acc));
+        const uint32_t codes = quant4(acc, sc);
+        // default caching: pass 2 reads the payload back right away
         *reinterpret_cast<uint32_t *>(ws_codes + base + e0) = codes;
-        if (lane_id() == 0) ws_scales[b] = s;
+        if (lane_id() == 0) ws_scales[b] = sc.s;
     }
 }
 
+// ReduceScatter, native: destination rank r = blockIdx.y.
 template <typename T, int NR, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 rs_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n) {
     constexpr int V = VecN<T>::n;
-    const size_t step = static_cast<size_t>(gridDim.x) * blockDim.x;
-    const size_t tid = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const size_t r = blockIdx.y;
     const size_t nvec = (m + V - 1) / V;
-    for (int r = 0; r < n; ++r) {
-        for (size_t v = tid; v < nvec; v += step) {
-            const size_t j0 = v * V;
-            const int valid = m - j0 < static_cast<size_t>(V) ? static_cast<int>(m - j0) : V;
-            float acc[V];
-            reduce_vec<T, NR, VEC>(send + r * m + j0, sstride, n, valid, acc);
-            storev<T, VEC>(recv + r * rstride + j0, valid, acc);
-        }
+    for (size_t v = thread_in_grid_x(); v < nvec; v += threads_in_grid_x()) {
+        const size_t j0 = v * V;
+        const int valid = m - j0 < static_cast<size_t>(V) ? static_cast<int>(m - j0) : V;
+        float acc[V];
+        reduce_vec<T, NR, VEC>(send + r * m + j0, sstride, n, valid, acc);
+        storev<T, VEC>(recv + r * rstride + j0, valid, acc);
     }
 }
 
+// ReduceScatter, FP8: destination rank r = blockIdx.y; blocks anchored at the
+// chunk start r*m.
 template <typename T, int NR, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 rs_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n) {
+    const size_t r = blockIdx.y;
     const size_t nbm = (m + kBlock - 1) / kBlock;
-    const size_t jobs = nbm * static_cast<size_t>(n);
     const int e0 = lane_id() * 4;
-    for (size_t job = global_warp(); job < jobs; job += num_warps()) {
-        const size_t r = job / nbm;
-        const size_t j0 = (job - r * nbm) * kBlock;
-        const int len = m - j0 < static_cast<size_t>(kBlock) ? static_cast<int>(m - j0) : kBlock;
-        const int valid = lane_valid(len);
+    for (size_t b = warp_in_grid_x(); b < nbm; b += warps_in_grid_x()) {
+        const size_t j0 = b * kBlock;
+        const int valid = lane_valid(j0, m);
         float acc[4];
         reduce_block_fp8<T, NR, VEC>(send + r * m + j0, sstride, n, valid, acc);
         store4<T, VEC>(recv + r * rstride + j0 + e0, valid, acc);
@@ -248,8 +246,10 @@ cudaError_t dispatch(rlx_dtype dtype, int n, bool vec, F &&f) {
 }
 
 template <typename K, typename... Args>
-cudaError_t launch(K kernel, size_t jobs, size_t jobs_per_cta, cudaStream_t stream, Args... args) {
-    const int grid = persistent_grid(reinterpret_cast<const void *>(kernel), jobs, jobs_per_cta);
+cudaError_t launch(K kernel, unsigned segments, size_t jobs_per_segment, size_t jobs_per_cta,
+                   cudaStream_t stream, Args... args) {
+    const dim3 grid = grid_2d(reinterpret_cast<const void *>(kernel), segments,
+                              jobs_per_segment, jobs_per_cta);
     kernel<<<grid, kThreads, 0, stream>>>(args...);
     return cudaGetLastError();
 }
@@ -266,11 +266,11 @@ cudaError_t launch_allreduce_flat(const void *send, void *recv, size_t count, si
         T *r = static_cast<T *>(recv);
         if (wire == RLX_WIRE_NATIVE) {
             const size_t nvec = (count + VecN<T>::n - 1) / VecN<T>::n;
-            return launch(flat_native_kernel<T, NR, VEC>, nvec, kThreads, stream, s, r, count,
+            return launch(flat_native_kernel<T, NR, VEC>, 1, nvec, kThreads, stream, s, r, count,
                           stride, nranks);
         }
         const size_t nblk = (count + kBlock - 1) / kBlock;
-        return launch(flat_fp8_kernel<T, NR, VEC>, nblk, kWarps, stream, s, r, count, stride,
+        return launch(flat_fp8_kernel<T, NR, VEC>, 1, nblk, kWarps, stream, s, r, count, stride,
                       nranks);
     });
 }
@@ -283,11 +283,12 @@ cudaError_t launch_tree_reduce(const void *send, void *recv, size_t count, size_
         const T *s = static_cast<const T *>(send);
         if (wire == RLX_WIRE_NATIVE) {
             const size_t nvec = (chunk + VecN<T>::n - 1) / VecN<T>::n;
-            return launch(tree_reduce_native_kernel<T, NR, VEC>, nvec, kThreads, stream, s,
-                          static_cast<T *>(recv), count, stride, nranks, chunk);
+            return launch(tree_reduce_native_kernel<T, NR, VEC>, static_cast<unsigned>(nranks),
+                          nvec, kThreads, stream, s, static_cast<T *>(recv), count, stride,
+                          nranks, chunk);
         }
         const size_t nblk = (count + kBlock - 1) / kBlock;
-        return launch(tree_reduce_fp8_kernel<T, NR, VEC>, nblk, kWarps, stream, s, count,
+        return launch(tree_reduce_fp8_kernel<T, NR, VEC>, 1, nblk, kWarps, stream, s, count,
                       stride, nranks, ws_codes, ws_scales);
     });
 }
@@ -298,13 +299,14 @@ cudaError_t launch_reduce_scatter(const void *send, size_t send_stride, void *re
     return dispatch(dtype, nranks, vec, [&]<typename T, int NR, bool VEC>() {
         const T *s = static_cast<const T *>(send);
         T *r = static_cast<T *>(recv);
+        const unsigned segs = static_cast<unsigned>(nranks);
         if (wire == RLX_WIRE_NATIVE) {
             const size_t nvec = (m + VecN<T>::n - 1) / VecN<T>::n;
-            return launch(rs_native_kernel<T, NR, VEC>, nvec, kThreads, stream, s, send_stride,
-                          r, recv_stride, m, nranks);
+            return launch(rs_native_kernel<T, NR, VEC>, segs, nvec, kThreads, stream, s,
+                          send_stride, r, recv_stride, m, nranks);
         }
-        const size_t jobs = (m + kBlock - 1) / kBlock * static_cast<size_t>(nranks);
-        return launch(rs_fp8_kernel<T, NR, VEC>, jobs, kWarps, stream, s, send_stride, r,
+        const size_t nbm = (m + kBlock - 1) / kBlock;
+        return launch(rs_fp8_kernel<T, NR, VEC>, segs, nbm, kWarps, stream, s, send_stride, r,
                       recv_stride, m, nranks);
     });
 }
