@@ -161,20 +161,20 @@ __device__ __forceinline__ void make_scales(const float (&amax)[K], Scale (&sc)[
 // Markstein's division theorem (P. Markstein, "Computation of elementary
 // functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1),
 // 1990): if y approximates 1/s with relative error below 2^-24 and q is a
-// faithful approximation of x/s, then r = x - s*q is exact and q + r*y
-// rounded to nearest is the correctly rounded quotient.  q0 = x*y can be up to
-// 1.5 ulp away, so one correction first makes it faithful, the second rounds
-// it correctly.  With s >= 2^-90 every residual that can affect an E4M3 code
-// (|x/s| >= 2^-10) is exact; smaller quotients only need their sign and a
-// magnitude below 2^-10, which the steps keep.  The sign is copied from x so
-// that x = -0 gives -0.
+// faithful approximation of x/s, then the residual s*q - x is exact and
+// q - (s*q - x)*y rounded to nearest is the correctly rounded quotient.
+// q0 = x*y can be up to 1.5 ulp away, so one correction first makes it
+// faithful, the second rounds it correctly.  With s >= 2^-90 every residual
+// that can affect an E4M3 code (|x/s| >= 2^-12) is exact; smaller quotients
+// keep their sign and a magnitude far below 2^-10, so their code (+-0) is
+// right.  The residual is taken as s*q - x (not x - s*q) so that x = -0
+// yields -0: the sum of an exact zero product and -0 is then -0.
 __device__ __forceinline__ float quotient_rn(float x, float s, float y) {
     float q = __fmul_rn(x, y);
-    float r = __fmaf_rn(-s, q, x);
-    q = __fmaf_rn(r, y, q);
-    r = __fmaf_rn(-s, q, x);
-    q = __fmaf_rn(r, y, q);
-    return copysignf(q, x);
+    float r = __fmaf_rn(s, q, -x);
+    q = __fmaf_rn(-r, y, q);
+    r = __fmaf_rn(s, q, -x);
+    return __fmaf_rn(-r, y, q);
 }
 
 // Quantise 4 values of a block with scale sc: code = e4m3_rne_sat(fl32(v/s));
@@ -233,6 +233,26 @@ __device__ __forceinline__ size_t thread_in_grid_x() {
 __device__ __forceinline__ size_t threads_in_grid_x() {
     return static_cast<size_t>(gridDim.x) * blockDim.x;
 }
+
+// Walks units first, first + step, first + 2*step, ... of a sequence of
+// equal segments (`per_seg` units each), segment-major, without dividing per
+// step: (seg, off) is the current unit.  Keeping all threads of a grid in the
+// same stretch of the sequence keeps the number of DRAM streams in flight
+// small.
+struct SegCursor {
+    size_t seg, off, per_seg, step_seg, step_off;
+    __device__ __forceinline__ SegCursor(size_t first, size_t step, size_t per_seg_)
+        : seg(first / per_seg_), off(first % per_seg_), per_seg(per_seg_),
+          step_seg(step / per_seg_), step_off(step % per_seg_) {}
+    __device__ __forceinline__ void next() {
+        off += step_off;
+        seg += step_seg;
+        if (off >= per_seg) {
+            off -= per_seg;
+            ++seg;
+        }
+    }
+};
 
 // Elements of a 128-block that belong to this lane: 0..4.
 __device__ __forceinline__ int lane_valid(size_t block_start, size_t len) {

@@ -13,7 +13,8 @@
 // flight.  On the FP8 wire a warp handles kJ consecutive 128-element blocks
 // at once (4 elements per lane per block): it reads them, applies
 // dequantise(quantise(.)) in registers and writes every destination.
-// Per-chunk work uses a 2-D grid (y = source rank, rank pair or chunk).
+// Chunked passes walk (chunk, unit) segment-major with a SegCursor, so all
+// warps stay within about one chunk (few DRAM streams open at a time).
 #include "rlx_device.cuh"
 #include "rlx_internal.h"
 
@@ -89,31 +90,37 @@ copy_kernel(const T *src, T *dst, size_t n) {
     }
 }
 
-// DDA-tree pass 2, native: chunk c = blockIdx.y of row c -> every other row.
+// DDA-tree pass 2, native: chunk c of row c -> chunk c of every other row.
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 tree_gather_native_kernel(T *recv, size_t count, size_t stride, int n, size_t chunk) {
-    const int c = blockIdx.y;
-    const size_t lo = static_cast<size_t>(c) * chunk;
-    if (lo >= count) return;
-    const size_t len = count - lo < chunk ? count - lo : chunk;
-    const size_t nvec = (len + kV<T> - 1) / kV<T>;
+    const size_t per = (chunk + kV<T> - 1) / kV<T>;
+    const size_t total = per * static_cast<size_t>(n);
     const size_t T_ = threads_in_grid_x();
-    const T *src = recv + c * stride + lo;
-    for (size_t v0 = thread_in_grid_x(); v0 < nvec; v0 += kUnroll * T_) {
+    SegCursor cur(thread_in_grid_x(), T_, per);
+    for (size_t g = thread_in_grid_x(); g < total; g += kUnroll * T_) {
         RawVec<T, VEC> a[kUnroll];
         int valid[kUnroll];
+        size_t c[kUnroll], i0[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            valid[u] = vec_valid<T>(v0 + u * T_, nvec, len);
-            if (valid[u]) a[u].load_cached(src + (v0 + u * T_) * kV<T>, valid[u]);
+            c[u] = cur.seg;
+            const size_t lo = cur.seg * chunk;
+            i0[u] = lo + cur.off * kV<T>;
+            valid[u] = 0;
+            if (g + u * T_ < total && i0[u] < count) {
+                const size_t hi = count - lo < chunk ? count : lo + chunk;
+                valid[u] = hi - i0[u] < static_cast<size_t>(kV<T>) ? static_cast<int>(hi - i0[u]) : kV<T>;
+                // the owner's chunk was just written by pass 1: default caching
+                a[u].load_cached(recv + c[u] * stride + i0[u], valid[u]);
+            }
+            cur.next();
         }
         for (int r = 0; r < n; ++r) {
-            if (r == c) continue;
-            T *dst = recv + r * stride + lo;
 #pragma unroll
             for (int u = 0; u < kUnroll; ++u)
-                if (valid[u]) a[u].store(dst + (v0 + u * T_) * kV<T>, valid[u]);
+                if (valid[u] && static_cast<size_t>(r) != c[u])
+                    a[u].store(recv + r * stride + i0[u], valid[u]);
         }
     }
 }
@@ -144,40 +151,47 @@ tree_gather_fp8_kernel(T *recv, size_t count, size_t stride, int n, const uint8_
     }
 }
 
-// AllGather, native: source rank s = blockIdx.y.
+// AllGather, native: unit = (source rank s, vector of its row).
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 ag_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n) {
-    const size_t s = blockIdx.y;
-    const size_t nvec = (m + kV<T> - 1) / kV<T>;
+    const size_t per = (m + kV<T> - 1) / kV<T>;
+    const size_t total = per * static_cast<size_t>(n);
     const size_t T_ = threads_in_grid_x();
-    const T *src = send + s * sstride;
-    for (size_t v0 = thread_in_grid_x(); v0 < nvec; v0 += kUnroll * T_) {
+    SegCursor cur(thread_in_grid_x(), T_, per);
+    for (size_t g = thread_in_grid_x(); g < total; g += kUnroll * T_) {
         RawVec<T, VEC> a[kUnroll];
         int valid[kUnroll];
+        size_t off[kUnroll];   // element offset within a destination row
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            valid[u] = vec_valid<T>(v0 + u * T_, nvec, m);
-            if (valid[u]) a[u].load(src + (v0 + u * T_) * kV<T>, valid[u]);
+            const size_t j0 = cur.off * kV<T>;
+            off[u] = cur.seg * m + j0;
+            valid[u] = g + u * T_ < total ? vec_valid<T>(cur.off, per, m) : 0;
+            if (valid[u]) a[u].load(send + cur.seg * sstride + j0, valid[u]);
+            cur.next();
         }
         for (int r = 0; r < n; ++r) {
-            T *dst = recv + r * rstride + s * m;
 #pragma unroll
             for (int u = 0; u < kUnroll; ++u)
-                if (valid[u]) a[u].store(dst + (v0 + u * T_) * kV<T>, valid[u]);
+                if (valid[u]) a[u].store(recv + r * rstride + off[u], valid[u]);
         }
     }
 }
 
-// AllGather, FP8: source rank s = blockIdx.y; blocks anchored at its row start.
+// AllGather, FP8: unit = (source rank s, group of kJ blocks of its row);
+// blocks anchored at the row start.
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 ag_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n) {
-    const size_t s = blockIdx.y;
     const size_t nbm = (m + kBlock - 1) / kBlock;
+    const size_t per = (nbm + kJ - 1) / kJ;
+    const size_t total = per * static_cast<size_t>(n);
     const int e0 = lane_id() * 4;
-    const T *src = send + s * sstride;
-    for (size_t b0 = warp_in_grid_x() * kJ; b0 < nbm; b0 += warps_in_grid_x() * kJ) {
+    SegCursor cur(warp_in_grid_x(), warps_in_grid_x(), per);
+    for (size_t g = warp_in_grid_x(); g < total; g += warps_in_grid_x(), cur.next()) {
+        const size_t s = cur.seg, b0 = cur.off * kJ;
+        const T *src = send + s * sstride;
         float v[kJ][4];
         int valid[kJ];
 #pragma unroll
@@ -194,40 +208,50 @@ ag_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, 
     }
 }
 
-// AlltoAll, native: pair = blockIdx.y = s * n + r moves chunk r of rank s to
-// chunk s of rank r.
+// AlltoAll, native: unit = (pair p = s*n + r, vector): chunk r of rank s goes
+// to chunk s of rank r.  Pairs in s-major order read each source row front
+// to back.
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 a2a_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n) {
-    const size_t s = blockIdx.y / n, r = blockIdx.y % n;
-    const T *src = send + s * sstride + r * m;
-    T *dst = recv + r * rstride + s * m;
-    const size_t nvec = (m + kV<T> - 1) / kV<T>;
+    const size_t per = (m + kV<T> - 1) / kV<T>;
+    const size_t nn = static_cast<size_t>(n);
+    const size_t total = per * nn * nn;
     const size_t T_ = threads_in_grid_x();
-    for (size_t v0 = thread_in_grid_x(); v0 < nvec; v0 += kUnroll * T_) {
+    SegCursor cur(thread_in_grid_x(), T_, per);
+    for (size_t g = thread_in_grid_x(); g < total; g += kUnroll * T_) {
         RawVec<T, VEC> a[kUnroll];
         int valid[kUnroll];
+        T *dst[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            valid[u] = vec_valid<T>(v0 + u * T_, nvec, m);
-            if (valid[u]) a[u].load(src + (v0 + u * T_) * kV<T>, valid[u]);
+            const size_t s = cur.seg / nn, r = cur.seg - s * nn, j0 = cur.off * kV<T>;
+            valid[u] = g + u * T_ < total ? vec_valid<T>(cur.off, per, m) : 0;
+            dst[u] = recv + r * rstride + s * m + j0;
+            if (valid[u]) a[u].load(send + s * sstride + r * m + j0, valid[u]);
+            cur.next();
         }
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u)
-            if (valid[u]) a[u].store(dst + (v0 + u * T_) * kV<T>, valid[u]);
+            if (valid[u]) a[u].store(dst[u], valid[u]);
     }
 }
 
-// AlltoAll, FP8: pair = blockIdx.y; blocks anchored at the chunk start r*m.
+// AlltoAll, FP8: unit = (pair, group of kJ blocks); blocks anchored at the
+// chunk start r*m.
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 a2a_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n) {
-    const size_t s = blockIdx.y / n, r = blockIdx.y % n;
-    const T *src = send + s * sstride + r * m;
-    T *dst = recv + r * rstride + s * m;
     const size_t nbm = (m + kBlock - 1) / kBlock;
+    const size_t per = (nbm + kJ - 1) / kJ;
+    const size_t nn = static_cast<size_t>(n);
+    const size_t total = per * nn * nn;
     const int e0 = lane_id() * 4;
-    for (size_t b0 = warp_in_grid_x() * kJ; b0 < nbm; b0 += warps_in_grid_x() * kJ) {
+    SegCursor cur(warp_in_grid_x(), warps_in_grid_x(), per);
+    for (size_t g = warp_in_grid_x(); g < total; g += warps_in_grid_x(), cur.next()) {
+        const size_t s = cur.seg / nn, r = cur.seg - s * nn, b0 = cur.off * kJ;
+        const T *src = send + s * sstride + r * m;
+        T *dst = recv + r * rstride + s * m;
         float v[kJ][4];
         int valid[kJ];
 #pragma unroll
@@ -281,9 +305,9 @@ cudaError_t launch_tree_gather(void *recv, size_t count, size_t stride, int nran
     return dispatch(dtype, vec, [&]<typename T, bool VEC>() {
         T *r = static_cast<T *>(recv);
         if (wire == RLX_WIRE_NATIVE)
-            return launch(tree_gather_native_kernel<T, VEC>, static_cast<unsigned>(nranks),
-                          nvec_of<T>(chunk), kThreads * kUnroll, stream, r, count, stride,
-                          nranks, chunk);
+            return launch(tree_gather_native_kernel<T, VEC>, 1,
+                          nvec_of<T>(chunk) * static_cast<size_t>(nranks), kThreads * kUnroll,
+                          stream, r, count, stride, nranks, chunk);
         return launch(tree_gather_fp8_kernel<T, VEC>, 1, nblk_of(count), kWarps * kJd, stream, r,
                       count, stride, nranks, ws_codes, ws_scales);
     });
@@ -295,11 +319,11 @@ cudaError_t launch_all_gather(const void *send, size_t send_stride, void *recv,
     return dispatch(dtype, vec, [&]<typename T, bool VEC>() {
         const T *s = static_cast<const T *>(send);
         T *r = static_cast<T *>(recv);
-        const unsigned segs = static_cast<unsigned>(nranks);
+        const size_t nn = static_cast<size_t>(nranks);
         if (wire == RLX_WIRE_NATIVE)
-            return launch(ag_native_kernel<T, VEC>, segs, nvec_of<T>(m), kThreads * kUnroll, stream,
-                          s, send_stride, r, recv_stride, m, nranks);
-        return launch(ag_fp8_kernel<T, VEC>, segs, nblk_of(m), kWarps * kJ, stream, s,
+            return launch(ag_native_kernel<T, VEC>, 1, nvec_of<T>(m) * nn, kThreads * kUnroll,
+                          stream, s, send_stride, r, recv_stride, m, nranks);
+        return launch(ag_fp8_kernel<T, VEC>, 1, nblk_of(m) * nn, kWarps * kJ, stream, s,
                       send_stride, r, recv_stride, m, nranks);
     });
 }
@@ -310,11 +334,11 @@ cudaError_t launch_alltoall(const void *send, size_t send_stride, void *recv,
     return dispatch(dtype, vec, [&]<typename T, bool VEC>() {
         const T *s = static_cast<const T *>(send);
         T *r = static_cast<T *>(recv);
-        const unsigned pairs = static_cast<unsigned>(nranks * nranks);
+        const size_t pairs = static_cast<size_t>(nranks) * static_cast<size_t>(nranks);
         if (wire == RLX_WIRE_NATIVE)
-            return launch(a2a_native_kernel<T, VEC>, pairs, nvec_of<T>(m), kThreads * kUnroll,
+            return launch(a2a_native_kernel<T, VEC>, 1, nvec_of<T>(m) * pairs, kThreads * kUnroll,
                           stream, s, send_stride, r, recv_stride, m, nranks);
-        return launch(a2a_fp8_kernel<T, VEC>, pairs, nblk_of(m), kWarps * kJ, stream, s,
+        return launch(a2a_fp8_kernel<T, VEC>, 1, nblk_of(m) * pairs, kWarps * kJ, stream, s,
                       send_stride, r, recv_stride, m, nranks);
     });
 }

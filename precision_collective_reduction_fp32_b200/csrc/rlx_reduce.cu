@@ -17,8 +17,9 @@
 //   FP8 wire: one warp per 128-element block, 4 elements per lane, so a block
 //     amax is one warp reduction; the warp loads the block from all N ranks,
 //     dequantises each rank's quantised block and sums in rank order.
-// Chunked passes use a 2-D grid (y = chunk / destination rank), so no thread
-// divides indices and every chunk gets the same share of the grid.
+// Chunked passes walk (chunk, unit) segment-major with a SegCursor: all warps
+// stay within about one chunk, which keeps few DRAM streams open, and no
+// index is divided per step.
 #include "rlx_device.cuh"
 #include "rlx_internal.h"
 
@@ -142,7 +143,7 @@ flat_native_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
 }
 
 template <typename T, int NR, bool VEC>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, NR <= 8 ? 3 : 1)
 flat_fp8_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
     const size_t nblk = (count + kBlock - 1) / kBlock;
     const int e0 = lane_id() * 4;
@@ -155,30 +156,31 @@ flat_fp8_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
     }
 }
 
-// DDA-tree pass 1, native: chunk c = blockIdx.y -> row c of recv.
+// DDA-tree pass 1, native: chunk c -> row c of recv.
 template <typename T, int NR, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 tree_reduce_native_kernel(const T *send, T *recv, size_t count, size_t stride, int n,
                           size_t chunk) {
     constexpr int V = VecN<T>::n;
-    const int c = blockIdx.y;
-    const size_t lo = static_cast<size_t>(c) * chunk;
-    if (lo >= count) return;
-    const size_t hi = count - lo < chunk ? count : lo + chunk;
-    const size_t nvec = (hi - lo + V - 1) / V;
-    for (size_t v = thread_in_grid_x(); v < nvec; v += threads_in_grid_x()) {
-        const size_t i0 = lo + v * V;
+    const size_t per = (chunk + V - 1) / V;
+    const size_t total = per * static_cast<size_t>(n);
+    SegCursor cur(thread_in_grid_x(), threads_in_grid_x(), per);
+    for (size_t g = thread_in_grid_x(); g < total; g += threads_in_grid_x(), cur.next()) {
+        const size_t lo = cur.seg * chunk;
+        const size_t i0 = lo + cur.off * V;
+        if (i0 >= count) continue;
+        const size_t hi = count - lo < chunk ? count : lo + chunk;
         const int valid = hi - i0 < static_cast<size_t>(V) ? static_cast<int>(hi - i0) : V;
         float acc[V];
         reduce_vec<T, NR, VEC>(send + i0, stride, n, valid, acc);
-        storev<T, VEC>(recv + c * stride + i0, valid, acc);
+        storev<T, VEC>(recv + cur.seg * stride + i0, valid, acc);
     }
 }
 
 // DDA-tree pass 1, FP8: reduce, then quantise the reduced block again into
 // the workspace payload (codes padded to whole blocks, one scale per block).
 template <typename T, int NR, bool VEC>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, NR <= 8 ? 3 : 1)
 tree_reduce_fp8_kernel(const T *send, size_t count, size_t stride, int n,
                        uint8_t *ws_codes, float *ws_scales) {
     const size_t nblk = (count + kBlock - 1) / kBlock;
@@ -195,15 +197,16 @@ tree_reduce_fp8_kernel(const T *send, size_t count, size_t stride, int n,
     }
 }
 
-// ReduceScatter, native: destination rank r = blockIdx.y.
+// ReduceScatter, native: unit = (destination rank r, vector of chunk r).
 template <typename T, int NR, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 rs_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n) {
     constexpr int V = VecN<T>::n;
-    const size_t r = blockIdx.y;
-    const size_t nvec = (m + V - 1) / V;
-    for (size_t v = thread_in_grid_x(); v < nvec; v += threads_in_grid_x()) {
-        const size_t j0 = v * V;
+    const size_t per = (m + V - 1) / V;
+    const size_t total = per * static_cast<size_t>(n);
+    SegCursor cur(thread_in_grid_x(), threads_in_grid_x(), per);
+    for (size_t g = thread_in_grid_x(); g < total; g += threads_in_grid_x(), cur.next()) {
+        const size_t r = cur.seg, j0 = cur.off * V;
         const int valid = m - j0 < static_cast<size_t>(V) ? static_cast<int>(m - j0) : V;
         float acc[V];
         reduce_vec<T, NR, VEC>(send + r * m + j0, sstride, n, valid, acc);
@@ -211,16 +214,17 @@ rs_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t 
     }
 }
 
-// ReduceScatter, FP8: destination rank r = blockIdx.y; blocks anchored at the
-// chunk start r*m.
+// ReduceScatter, FP8: unit = (destination rank r, 128-block of chunk r);
+// blocks anchored at the chunk start r*m.
 template <typename T, int NR, bool VEC>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, NR <= 8 ? 3 : 1)
 rs_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n) {
-    const size_t r = blockIdx.y;
-    const size_t nbm = (m + kBlock - 1) / kBlock;
+    const size_t per = (m + kBlock - 1) / kBlock;
+    const size_t total = per * static_cast<size_t>(n);
     const int e0 = lane_id() * 4;
-    for (size_t b = warp_in_grid_x(); b < nbm; b += warps_in_grid_x()) {
-        const size_t j0 = b * kBlock;
+    SegCursor cur(warp_in_grid_x(), warps_in_grid_x(), per);
+    for (size_t g = warp_in_grid_x(); g < total; g += warps_in_grid_x(), cur.next()) {
+        const size_t r = cur.seg, j0 = cur.off * kBlock;
         const int valid = lane_valid(j0, m);
         float acc[4];
         reduce_block_fp8<T, NR, VEC>(send + r * m + j0, sstride, n, valid, acc);
@@ -283,9 +287,9 @@ cudaError_t launch_tree_reduce(const void *send, void *recv, size_t count, size_
         const T *s = static_cast<const T *>(send);
         if (wire == RLX_WIRE_NATIVE) {
             const size_t nvec = (chunk + VecN<T>::n - 1) / VecN<T>::n;
-            return launch(tree_reduce_native_kernel<T, NR, VEC>, static_cast<unsigned>(nranks),
-                          nvec, kThreads, stream, s, static_cast<T *>(recv), count, stride,
-                          nranks, chunk);
+            return launch(tree_reduce_native_kernel<T, NR, VEC>, 1,
+                          nvec * static_cast<size_t>(nranks), kThreads, stream, s,
+                          static_cast<T *>(recv), count, stride, nranks, chunk);
         }
         const size_t nblk = (count + kBlock - 1) / kBlock;
         return launch(tree_reduce_fp8_kernel<T, NR, VEC>, 1, nblk, kWarps, stream, s, count,
@@ -299,14 +303,14 @@ cudaError_t launch_reduce_scatter(const void *send, size_t send_stride, void *re
     return dispatch(dtype, nranks, vec, [&]<typename T, int NR, bool VEC>() {
         const T *s = static_cast<const T *>(send);
         T *r = static_cast<T *>(recv);
-        const unsigned segs = static_cast<unsigned>(nranks);
+        const size_t nn = static_cast<size_t>(nranks);
         if (wire == RLX_WIRE_NATIVE) {
             const size_t nvec = (m + VecN<T>::n - 1) / VecN<T>::n;
-            return launch(rs_native_kernel<T, NR, VEC>, segs, nvec, kThreads, stream, s,
+            return launch(rs_native_kernel<T, NR, VEC>, 1, nvec * nn, kThreads, stream, s,
                           send_stride, r, recv_stride, m, nranks);
         }
         const size_t nbm = (m + kBlock - 1) / kBlock;
-        return launch(rs_fp8_kernel<T, NR, VEC>, segs, nbm, kWarps, stream, s, send_stride, r,
+        return launch(rs_fp8_kernel<T, NR, VEC>, 1, nbm * nn, kWarps, stream, s, send_stride, r,
                       recv_stride, m, nranks);
     });
 }
