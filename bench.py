@@ -176,44 +176,48 @@ class Step:
     """Device buffers for one batch and the twelve operations of one step,
     each issued through the C ABI (librlx.so) on the current stream."""
 
-    def __init__(self, x_host: np.ndarray, device):
+    def __init__(self, x_host: np.ndarray, device, pad: int = 0):
         import torch
         from precision_collective_reduction_fp32_b200 import binding as B
         self.B, self.torch = B, torch
         n, c = x_host.shape
         self.n, self.c, self.m = n, c, c // n
+        # rank rows are `pitch` elements apart (pad > 0 breaks power-of-two
+        # distances between the rows that are streamed together)
+        self.pitch, self.mpitch = c + pad, self.m + pad
         t = lambda *s, dt=torch.float32: torch.empty(*s, dtype=dt, device=device)
-        self.x = torch.from_numpy(x_host).to(device)
-        self.out = t((n, c))
-        self.y = t((n, c))
-        self.codes = t((n, c), dt=torch.uint8)
+        self.x = t((n, self.pitch))
+        self.x[:, :c].copy_(torch.from_numpy(x_host))
+        self.out = t((n, self.pitch))
+        self.y = t((n, self.pitch))
+        self.codes = t((n, self.pitch), dt=torch.uint8)
         self.scales = t((n, (c + BLOCK - 1) // BLOCK))
-        self.rs = t((n, self.m))
+        self.rs = t((n, self.mpitch))
         self.ws_bytes = B.rlx_workspace_bytes(B.RLX_COLL_ALLREDUCE_TREE, c, n, B.RLX_F32,
                                               B.RLX_WIRE_FP8_E4M3)
         self.ws = t((self.ws_bytes,), dt=torch.uint8)
 
     def ops(self, stream):
-        B, n, c, m = self.B, self.n, self.c, self.m
+        B, n, c, m, p, mp = self.B, self.n, self.c, self.m, self.pitch, self.mpitch
         x, out, y, rs = self.x.data_ptr(), self.out.data_ptr(), self.y.data_ptr(), self.rs.data_ptr()
         F, NAT, FP8 = B.RLX_F32, B.RLX_WIRE_NATIVE, B.RLX_WIRE_FP8_E4M3
         return [
-            ("quantize_fp8", lambda: B.rlx_quantize_fp8(x, F, n, c, c, self.codes.data_ptr(),
+            ("quantize_fp8", lambda: B.rlx_quantize_fp8(x, F, n, c, p, self.codes.data_ptr(),
                                                         self.scales.data_ptr(), stream)),
             ("dequantize_fp8", lambda: B.rlx_dequantize_fp8(self.codes.data_ptr(), self.scales.data_ptr(),
-                                                            n, c, c, y, F, stream)),
-            ("allreduce_flat_native", lambda: B.rlx_allreduce_flat(x, out, c, c, n, F, NAT, B.RLX_SUM, stream)),
-            ("allreduce_flat_fp8", lambda: B.rlx_allreduce_flat(x, out, c, c, n, F, FP8, B.RLX_SUM, stream)),
-            ("allreduce_tree_native", lambda: B.rlx_allreduce_tree(x, out, c, c, n, F, NAT, B.RLX_SUM,
+                                                            n, c, p, y, F, stream)),
+            ("allreduce_flat_native", lambda: B.rlx_allreduce_flat(x, out, c, p, n, F, NAT, B.RLX_SUM, stream)),
+            ("allreduce_flat_fp8", lambda: B.rlx_allreduce_flat(x, out, c, p, n, F, FP8, B.RLX_SUM, stream)),
+            ("allreduce_tree_native", lambda: B.rlx_allreduce_tree(x, out, c, p, n, F, NAT, B.RLX_SUM,
                                                                    None, 0, stream)),
-            ("allreduce_tree_fp8", lambda: B.rlx_allreduce_tree(x, out, c, c, n, F, FP8, B.RLX_SUM,
+            ("allreduce_tree_fp8", lambda: B.rlx_allreduce_tree(x, out, c, p, n, F, FP8, B.RLX_SUM,
                                                                 self.ws.data_ptr(), self.ws_bytes, stream)),
-            ("reduce_scatter_native", lambda: B.rlx_reduce_scatter(x, c, rs, m, m, n, F, NAT, B.RLX_SUM, stream)),
-            ("reduce_scatter_fp8", lambda: B.rlx_reduce_scatter(x, c, rs, m, m, n, F, FP8, B.RLX_SUM, stream)),
-            ("all_gather_native", lambda: B.rlx_all_gather(rs, m, y, c, m, n, F, NAT, stream)),
-            ("all_gather_fp8", lambda: B.rlx_all_gather(rs, m, y, c, m, n, F, FP8, stream)),
-            ("alltoall_native", lambda: B.rlx_alltoall(x, c, y, c, m, n, F, NAT, stream)),
-            ("alltoall_fp8", lambda: B.rlx_alltoall(x, c, y, c, m, n, F, FP8, stream)),
+            ("reduce_scatter_native", lambda: B.rlx_reduce_scatter(x, p, rs, mp, m, n, F, NAT, B.RLX_SUM, stream)),
+            ("reduce_scatter_fp8", lambda: B.rlx_reduce_scatter(x, p, rs, mp, m, n, F, FP8, B.RLX_SUM, stream)),
+            ("all_gather_native", lambda: B.rlx_all_gather(rs, mp, y, p, m, n, F, NAT, stream)),
+            ("all_gather_fp8", lambda: B.rlx_all_gather(rs, mp, y, p, m, n, F, FP8, stream)),
+            ("alltoall_native", lambda: B.rlx_alltoall(x, p, y, p, m, n, F, NAT, stream)),
+            ("alltoall_fp8", lambda: B.rlx_alltoall(x, p, y, p, m, n, F, FP8, stream)),
         ]
 
 
@@ -280,20 +284,21 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
     host_in = torch.from_numpy(x_host).pin_memory()
     host_out = torch.empty((NRANKS, count), dtype=torch.float32).pin_memory()
     Ke = max(1, min(K, args.e2e_steps))
+    x_dev, out_dev = step.x[:, :count], step.out[:, :count]
     for _ in range(2):
-        step.x.copy_(host_in, non_blocking=True)
+        x_dev.copy_(host_in, non_blocking=True)
         for _, f in ops:
             f()
-        host_out.copy_(step.out, non_blocking=True)
+        host_out.copy_(out_dev, non_blocking=True)
     torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(Ke):
-        step.x.copy_(host_in, non_blocking=True)
+        x_dev.copy_(host_in, non_blocking=True)
         for _, f in ops:
             f()
-        host_out.copy_(step.out, non_blocking=True)   # the FP8 tree allreduce result
+        host_out.copy_(out_dev, non_blocking=True)   # the FP8 tree allreduce result
     e1.record(stream)
     torch.cuda.synchronize()
     e_dev = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)

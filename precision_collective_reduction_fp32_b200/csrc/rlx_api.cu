@@ -11,14 +11,20 @@
 
 namespace rlx {
 
-dim3 grid_2d(const void *kernel, unsigned segments, size_t jobs_per_segment,
-             size_t jobs_per_cta) {
-    static std::mutex mu;
-    static std::map<std::pair<int, const void *>, int> cap_cache;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    int cap = 0;
-    {
+dim3 grid_for(const void *kernel, size_t units, size_t units_per_cta) {
+    if (units >= (size_t{1} << 32)) return dim3(0, 1, 1);
+    size_t x = (units + units_per_cta - 1) / units_per_cta;
+    if (x == 0) x = 1;
+#ifndef RLX_GRID_WAVES
+#define RLX_GRID_WAVES 0
+#endif
+    // RLX_GRID_WAVES > 0 caps the grid at that many waves of resident CTAs.
+    if (RLX_GRID_WAVES > 0) {
+        static std::mutex mu;
+        static std::map<std::pair<int, const void *>, int> cap_cache;
+        int dev = 0;
+        cudaGetDevice(&dev);
+        int cap = 0;
         std::lock_guard<std::mutex> lock(mu);
         auto it = cap_cache.find({dev, kernel});
         if (it != cap_cache.end()) {
@@ -28,17 +34,13 @@ dim3 grid_2d(const void *kernel, unsigned segments, size_t jobs_per_segment,
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0);
             cap = sms * (per_sm > 0 ? per_sm : 1);
-            if (cap <= 0) cap = 1;
             cap_cache[{dev, kernel}] = cap;
         }
+        const size_t lim = static_cast<size_t>(cap) * RLX_GRID_WAVES;
+        if (lim > 0 && x > lim) x = lim;
     }
-    if (segments == 0) segments = 1;
-    size_t need = (jobs_per_segment + jobs_per_cta - 1) / jobs_per_cta;
-    if (need == 0) need = 1;
-    size_t share = (static_cast<size_t>(cap) + segments - 1) / segments;
-    if (share == 0) share = 1;
-    const size_t x = need < share ? need : share;
-    return dim3(static_cast<unsigned>(x), segments, 1);
+    if (x > 0x7fffffffu) x = 0x7fffffffu;
+    return dim3(static_cast<unsigned>(x), 1, 1);
 }
 
 }  // namespace rlx

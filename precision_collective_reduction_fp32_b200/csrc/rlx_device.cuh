@@ -34,18 +34,45 @@ __device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
     return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
 
-// Element traits: load/store one element as fp32 (streaming cache hints).
+// Cache policy of the streaming loads and stores (inputs are read once,
+// outputs written once): RLX_LD_CS / RLX_ST_CS = 1 use the evict-first
+// ".cs" forms, 0 the default write-back forms.
+#ifndef RLX_LD_CS
+#define RLX_LD_CS 1
+#endif
+#ifndef RLX_ST_CS
+#define RLX_ST_CS 1
+#endif
+
+template <typename V>
+__device__ __forceinline__ V ld_stream(const V *p) {
+#if RLX_LD_CS
+    return __ldcs(p);
+#else
+    return *p;
+#endif
+}
+template <typename V>
+__device__ __forceinline__ void st_stream(V *p, V v) {
+#if RLX_ST_CS
+    __stcs(p, v);
+#else
+    *p = v;
+#endif
+}
+
+// Element traits: load/store one element as fp32.
 template <typename T> struct Elem;
 template <> struct Elem<float> {
-    __device__ __forceinline__ static float load(const float *p) { return __ldcs(p); }
-    __device__ __forceinline__ static void store(float *p, float v) { __stcs(p, v); }
+    __device__ __forceinline__ static float load(const float *p) { return ld_stream(p); }
+    __device__ __forceinline__ static void store(float *p, float v) { st_stream(p, v); }
 };
 template <> struct Elem<uint16_t> {  // bf16 bit patterns
     __device__ __forceinline__ static float load(const uint16_t *p) {
-        return bf16_bits_to_f32(__ldcs(reinterpret_cast<const unsigned short *>(p)));
+        return bf16_bits_to_f32(ld_stream(reinterpret_cast<const unsigned short *>(p)));
     }
     __device__ __forceinline__ static void store(uint16_t *p, float v) {
-        __stcs(reinterpret_cast<unsigned short *>(p), f32_to_bf16_bits(v));
+        st_stream(reinterpret_cast<unsigned short *>(p), f32_to_bf16_bits(v));
     }
 };
 
@@ -55,10 +82,10 @@ template <typename T, bool VEC>
 __device__ __forceinline__ void load4(const T *p, int valid, float (&v)[4]) {
     if (VEC && valid == 4) {
         if constexpr (sizeof(T) == 4) {
-            const float4 q = __ldcs(reinterpret_cast<const float4 *>(p));
+            const float4 q = ld_stream(reinterpret_cast<const float4 *>(p));
             v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
         } else {
-            const uint2 q = __ldcs(reinterpret_cast<const uint2 *>(p));
+            const uint2 q = ld_stream(reinterpret_cast<const uint2 *>(p));
             v[0] = __uint_as_float(q.x << 16);
             v[1] = __uint_as_float(q.x & 0xffff0000u);
             v[2] = __uint_as_float(q.y << 16);
@@ -74,14 +101,14 @@ template <typename T, bool VEC>
 __device__ __forceinline__ void store4(T *p, int valid, const float (&v)[4]) {
     if (VEC && valid == 4) {
         if constexpr (sizeof(T) == 4) {
-            __stcs(reinterpret_cast<float4 *>(p), make_float4(v[0], v[1], v[2], v[3]));
+            st_stream(reinterpret_cast<float4 *>(p), make_float4(v[0], v[1], v[2], v[3]));
         } else {
             uint2 q;
             q.x = static_cast<uint32_t>(f32_to_bf16_bits(v[0])) |
                   (static_cast<uint32_t>(f32_to_bf16_bits(v[1])) << 16);
             q.y = static_cast<uint32_t>(f32_to_bf16_bits(v[2])) |
                   (static_cast<uint32_t>(f32_to_bf16_bits(v[3])) << 16);
-            __stcs(reinterpret_cast<uint2 *>(p), q);
+            st_stream(reinterpret_cast<uint2 *>(p), q);
         }
     } else {
 #pragma unroll
@@ -218,41 +245,55 @@ __device__ __forceinline__ void wire_fp8_blocks(float (&v)[K][4]) {
     for (int k = 0; k < K; ++k) dequant4(quant4(v[k], sc[k]), sc[k].s, v[k]);
 }
 
-// ----------------------------------------------------------- grid helpers
+// ----------------------------------------------------------- work layout
 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
-__device__ __forceinline__ size_t warp_in_grid_x() {
-    return (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+
+// n / d for 32-bit n by a multiply and shifts (T. Granlund, P. Montgomery,
+// "Division by invariant integers using multiplication", PLDI 1994, sec. 4):
+// with l = ceil(log2 d), m = floor(2^32 (2^l - d) / d) + 1,
+// q = (t + ((n - t) >> min(l,1))) >> max(l-1,0), t = mulhi(m, n).
+struct FastDiv {
+    uint32_t d, m, s1, s2;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+    uint32_t l = 0;
+    while (l < 32 && (uint64_t{1} << l) < d) ++l;
+    FastDiv f;
+    f.d = d;
+    f.m = static_cast<uint32_t>((((uint64_t{1} << l) - d) << 32) / d + 1);
+    f.s1 = l < 1 ? l : 1;
+    f.s2 = l > 0 ? l - 1 : 0;
+    return f;
 }
-__device__ __forceinline__ size_t warps_in_grid_x() {
-    return (static_cast<size_t>(gridDim.x) * blockDim.x) >> 5;
-}
-__device__ __forceinline__ size_t thread_in_grid_x() {
-    return static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-}
-__device__ __forceinline__ size_t threads_in_grid_x() {
-    return static_cast<size_t>(gridDim.x) * blockDim.x;
+__host__ __device__ __forceinline__ uint32_t fast_div(uint32_t n, const FastDiv &f) {
+#ifdef __CUDA_ARCH__
+    const uint32_t t = __umulhi(f.m, n);
+#else
+    const uint32_t t = static_cast<uint32_t>((static_cast<uint64_t>(f.m) * n) >> 32);
+#endif
+    return (t + ((n - t) >> f.s1)) >> f.s2;
 }
 
-// Walks units first, first + step, first + 2*step, ... of a sequence of
-// equal segments (`per_seg` units each), segment-major, without dividing per
-// step: (seg, off) is the current unit.  Keeping all threads of a grid in the
-// same stretch of the sequence keeps the number of DRAM streams in flight
-// small.
-struct SegCursor {
-    size_t seg, off, per_seg, step_seg, step_off;
-    __device__ __forceinline__ SegCursor(size_t first, size_t step, size_t per_seg_)
-        : seg(first / per_seg_), off(first % per_seg_), per_seg(per_seg_),
-          step_seg(step / per_seg_), step_off(step % per_seg_) {}
-    __device__ __forceinline__ void next() {
-        off += step_off;
-        seg += step_seg;
-        if (off >= per_seg) {
-            off -= per_seg;
-            ++seg;
+// Units of work of the calling warp.  The grid covers units 0..total-1 in
+// order: CTA b owns units [b*W*P, (b+1)*W*P) (W warps per CTA) and its warps
+// take them round-robin, P per warp; a grid smaller than that loops.  CTAs
+// are started in index order, so the CTAs resident at any moment work on one
+// compact stretch of the data, which keeps few DRAM pages open.  f(g) is
+// called with the same g by all 32 lanes.
+template <int P, typename F>
+__device__ __forceinline__ void for_each_unit(uint32_t total, F &&f) {
+    constexpr uint32_t W = 256 / 32;   // rlx kernels run 256-thread CTAs
+    const uint32_t w = threadIdx.x >> 5;
+    const size_t span = static_cast<size_t>(W) * P;
+    for (size_t base = blockIdx.x * span; base < total; base += gridDim.x * span) {
+#pragma unroll 1
+        for (int p = 0; p < P; ++p) {
+            const size_t g = base + static_cast<size_t>(p) * W + w;
+            if (g < total) f(static_cast<uint32_t>(g));
         }
     }
-};
+}
 
 // Elements of a 128-block that belong to this lane: 0..4.
 __device__ __forceinline__ int lane_valid(size_t block_start, size_t len) {

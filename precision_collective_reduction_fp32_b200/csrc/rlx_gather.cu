@@ -9,21 +9,40 @@
 // quantises what it sends and the receiver dequantises it.
 //
 // On the native wire these passes move bytes only (16-byte vectors, no
-// conversion), so results are bit copies; each thread keeps kUnroll vectors in
-// flight.  On the FP8 wire a warp handles kJ consecutive 128-element blocks
+// conversion), so results are bit copies; a warp moves kUnroll x 512
+// contiguous bytes per step (lane l takes vectors l, l+32, ...), so each of
+// its stores to a destination row continues the previous one.  On the FP8 wire a warp handles kJ consecutive 128-element blocks
 // at once (4 elements per lane per block): it reads them, applies
 // dequantise(quantise(.)) in registers and writes every destination.
-// Chunked passes walk (chunk, unit) segment-major with a SegCursor, so all
-// warps stay within about one chunk (few DRAM streams open at a time).
+// Units of work are numbered in memory order (segment-major) and handed out
+// in CTA-sized runs by for_each_unit, so the CTAs in flight stream one
+// compact stretch of the data.
 #include "rlx_device.cuh"
 #include "rlx_internal.h"
 
 namespace rlx {
 namespace {
 
-constexpr int kUnroll = 4;  // 16-byte vectors in flight per thread (native copies)
-constexpr int kJ = 4;       // 128-blocks in flight per warp (FP8 single-source)
-constexpr int kJd = 8;      // 128-blocks per warp when reading FP8 payloads
+#ifndef RLX_UNROLL
+#define RLX_UNROLL 4
+#endif
+#ifndef RLX_J
+#define RLX_J 4
+#endif
+#ifndef RLX_JD
+#define RLX_JD 8
+#endif
+constexpr int kUnroll = RLX_UNROLL;  // 16-byte vectors per lane in flight (native copies)
+constexpr int kJ = RLX_J;            // 128-blocks in flight per warp (FP8 single-source)
+constexpr int kJd = RLX_JD;          // 128-blocks per warp when reading FP8 payloads
+#ifndef RLX_P_COPY
+#define RLX_P_COPY 1
+#endif
+#ifndef RLX_P_GFP8
+#define RLX_P_GFP8 1
+#endif
+constexpr int kPc = RLX_P_COPY;      // units per warp per CTA run, native copies
+constexpr int kPg = RLX_P_GFP8;      // units per warp per CTA run, FP8 passes
 
 template <typename T> constexpr int kV = 16 / sizeof(T);
 
@@ -34,7 +53,7 @@ struct RawVec {
     T e[kV<T>];
     __device__ __forceinline__ void load(const T *p, int valid) {
         if (VEC && valid == kV<T>) {
-            q = __ldcs(reinterpret_cast<const uint4 *>(p));
+            q = ld_stream(reinterpret_cast<const uint4 *>(p));
         } else {
 #pragma unroll
             for (int k = 0; k < kV<T>; ++k)
@@ -53,7 +72,7 @@ struct RawVec {
     }
     __device__ __forceinline__ void store(T *p, int valid) const {
         if (VEC && valid == kV<T>) {
-            __stcs(reinterpret_cast<uint4 *>(p), q);
+            st_stream(reinterpret_cast<uint4 *>(p), q);
         } else {
 #pragma unroll
             for (int k = 0; k < kV<T>; ++k)
@@ -71,68 +90,79 @@ __device__ __forceinline__ int vec_valid(size_t v, size_t nvec, size_t len) {
 
 // ------------------------------------------------------------------ kernels
 
+// Vectors of one unit: unit u of a segment covers vectors
+// [u*32*kUnroll, (u+1)*32*kUnroll); lane l takes u*32*kUnroll + k*32 + l, so
+// each warp store continues the previous one.
+constexpr int kWarpVecs = 32 * kUnroll;
+
+// Loads the unit's vectors of a segment of `len` elements at `src`.
+template <typename T, bool VEC, bool CACHED = false>
+__device__ __forceinline__ void load_unit(const T *src, size_t unit, size_t len,
+                                          RawVec<T, VEC> (&a)[kUnroll], int (&valid)[kUnroll]) {
+    const size_t nv = (len + kV<T> - 1) / kV<T>;
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const size_t v = unit * kWarpVecs + u * 32 + lane_id();
+        valid[u] = vec_valid<T>(v, nv, len);
+        if (valid[u]) {
+            if (CACHED) a[u].load_cached(src + v * kV<T>, valid[u]);
+            else a[u].load(src + v * kV<T>, valid[u]);
+        }
+    }
+}
+
+template <typename T, bool VEC>
+__device__ __forceinline__ void store_unit(T *dst, size_t unit, const RawVec<T, VEC> (&a)[kUnroll],
+                                           const int (&valid)[kUnroll]) {
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u)
+        if (valid[u]) a[u].store(dst + (unit * kWarpVecs + u * 32 + lane_id()) * kV<T>, valid[u]);
+}
+
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 copy_kernel(const T *src, T *dst, size_t n) {
-    const size_t nvec = (n + kV<T> - 1) / kV<T>;
-    const size_t T_ = threads_in_grid_x();
-    for (size_t v0 = thread_in_grid_x(); v0 < nvec; v0 += kUnroll * T_) {
+    const uint32_t units = static_cast<uint32_t>(((n + kV<T> - 1) / kV<T> + kWarpVecs - 1) / kWarpVecs);
+    for_each_unit<kPc>(units, [&](uint32_t g) {
         RawVec<T, VEC> a[kUnroll];
         int valid[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            valid[u] = vec_valid<T>(v0 + u * T_, nvec, n);
-            if (valid[u]) a[u].load(src + (v0 + u * T_) * kV<T>, valid[u]);
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u)
-            if (valid[u]) a[u].store(dst + (v0 + u * T_) * kV<T>, valid[u]);
-    }
+        load_unit<T, VEC>(src, g, n, a, valid);
+        store_unit<T, VEC>(dst, g, a, valid);
+    });
 }
 
-// DDA-tree pass 2, native: chunk c of row c -> chunk c of every other row.
+// DDA-tree pass 2, native: unit = (chunk c, unit of it); chunk c of row c ->
+// chunk c of every other row.
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
-tree_gather_native_kernel(T *recv, size_t count, size_t stride, int n, size_t chunk) {
-    const size_t per = (chunk + kV<T> - 1) / kV<T>;
-    const size_t total = per * static_cast<size_t>(n);
-    const size_t T_ = threads_in_grid_x();
-    SegCursor cur(thread_in_grid_x(), T_, per);
-    for (size_t g = thread_in_grid_x(); g < total; g += kUnroll * T_) {
+tree_gather_native_kernel(T *recv, size_t count, size_t stride, int n, size_t chunk,
+                          FastDiv per_chunk) {
+    const uint32_t units = per_chunk.d * static_cast<uint32_t>(n);
+    for_each_unit<kPc>(units, [&](uint32_t g) {
+        const uint32_t c = fast_div(g, per_chunk);
+        const size_t lo = static_cast<size_t>(c) * chunk;
+        if (lo >= count) return;
+        const size_t len = count - lo < chunk ? count - lo : chunk;
+        const size_t unit = g - c * per_chunk.d;
         RawVec<T, VEC> a[kUnroll];
         int valid[kUnroll];
-        size_t c[kUnroll], i0[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            c[u] = cur.seg;
-            const size_t lo = cur.seg * chunk;
-            i0[u] = lo + cur.off * kV<T>;
-            valid[u] = 0;
-            if (g + u * T_ < total && i0[u] < count) {
-                const size_t hi = count - lo < chunk ? count : lo + chunk;
-                valid[u] = hi - i0[u] < static_cast<size_t>(kV<T>) ? static_cast<int>(hi - i0[u]) : kV<T>;
-                // the owner's chunk was just written by pass 1: default caching
-                a[u].load_cached(recv + c[u] * stride + i0[u], valid[u]);
-            }
-            cur.next();
-        }
-        for (int r = 0; r < n; ++r) {
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u)
-                if (valid[u] && static_cast<size_t>(r) != c[u])
-                    a[u].store(recv + r * stride + i0[u], valid[u]);
-        }
-    }
+        // the owner's chunk was just written by pass 1: default caching
+        load_unit<T, VEC, true>(recv + c * stride + lo, unit, len, a, valid);
+        for (int r = 0; r < n; ++r)
+            if (static_cast<uint32_t>(r) != c) store_unit<T, VEC>(recv + r * stride + lo, unit, a, valid);
+    });
 }
 
-// DDA-tree pass 2, FP8: dequantise the payload blocks into every row.
+// DDA-tree pass 2, FP8: unit = kJd payload blocks, dequantised into every row.
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 tree_gather_fp8_kernel(T *recv, size_t count, size_t stride, int n, const uint8_t *ws_codes,
                        const float *ws_scales) {
     const size_t nblk = (count + kBlock - 1) / kBlock;
+    const uint32_t units = static_cast<uint32_t>((nblk + kJd - 1) / kJd);
     const int e0 = lane_id() * 4;
-    for (size_t b0 = warp_in_grid_x() * kJd; b0 < nblk; b0 += warps_in_grid_x() * kJd) {
+    for_each_unit<kPg>(units, [&](uint32_t g) {
+        const size_t b0 = static_cast<size_t>(g) * kJd;
         float y[kJd][4];
         int valid[kJd];
 #pragma unroll
@@ -148,49 +178,36 @@ tree_gather_fp8_kernel(T *recv, size_t count, size_t stride, int n, const uint8_
 #pragma unroll
             for (int j = 0; j < kJd; ++j)
                 store4<T, VEC>(recv + r * stride + (b0 + j) * kBlock + e0, valid[j], y[j]);
-    }
+    });
 }
 
-// AllGather, native: unit = (source rank s, vector of its row).
+// AllGather, native: unit = (source rank s, unit of its row).
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
-ag_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n) {
-    const size_t per = (m + kV<T> - 1) / kV<T>;
-    const size_t total = per * static_cast<size_t>(n);
-    const size_t T_ = threads_in_grid_x();
-    SegCursor cur(thread_in_grid_x(), T_, per);
-    for (size_t g = thread_in_grid_x(); g < total; g += kUnroll * T_) {
+ag_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n,
+                 FastDiv per_row) {
+    const uint32_t units = per_row.d * static_cast<uint32_t>(n);
+    for_each_unit<kPc>(units, [&](uint32_t g) {
+        const uint32_t s = fast_div(g, per_row);
+        const size_t unit = g - s * per_row.d;
         RawVec<T, VEC> a[kUnroll];
         int valid[kUnroll];
-        size_t off[kUnroll];   // element offset within a destination row
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const size_t j0 = cur.off * kV<T>;
-            off[u] = cur.seg * m + j0;
-            valid[u] = g + u * T_ < total ? vec_valid<T>(cur.off, per, m) : 0;
-            if (valid[u]) a[u].load(send + cur.seg * sstride + j0, valid[u]);
-            cur.next();
-        }
-        for (int r = 0; r < n; ++r) {
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u)
-                if (valid[u]) a[u].store(recv + r * rstride + off[u], valid[u]);
-        }
-    }
+        load_unit<T, VEC>(send + s * sstride, unit, m, a, valid);
+        for (int r = 0; r < n; ++r) store_unit<T, VEC>(recv + r * rstride + s * m, unit, a, valid);
+    });
 }
 
-// AllGather, FP8: unit = (source rank s, group of kJ blocks of its row);
-// blocks anchored at the row start.
+// AllGather, FP8: unit = (source rank s, kJ blocks of its row); blocks
+// anchored at the row start.
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
-ag_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n) {
-    const size_t nbm = (m + kBlock - 1) / kBlock;
-    const size_t per = (nbm + kJ - 1) / kJ;
-    const size_t total = per * static_cast<size_t>(n);
+ag_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n,
+              FastDiv per_row) {
+    const uint32_t units = per_row.d * static_cast<uint32_t>(n);
     const int e0 = lane_id() * 4;
-    SegCursor cur(warp_in_grid_x(), warps_in_grid_x(), per);
-    for (size_t g = warp_in_grid_x(); g < total; g += warps_in_grid_x(), cur.next()) {
-        const size_t s = cur.seg, b0 = cur.off * kJ;
+    for_each_unit<kPg>(units, [&](uint32_t g) {
+        const uint32_t s = fast_div(g, per_row);
+        const size_t b0 = static_cast<size_t>(g - s * per_row.d) * kJ;
         const T *src = send + s * sstride;
         float v[kJ][4];
         int valid[kJ];
@@ -205,53 +222,41 @@ ag_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, 
 #pragma unroll
             for (int j = 0; j < kJ; ++j) store4<T, VEC>(dst + (b0 + j) * kBlock + e0, valid[j], v[j]);
         }
-    }
+    });
 }
 
-// AlltoAll, native: unit = (pair p = s*n + r, vector): chunk r of rank s goes
-// to chunk s of rank r.  Pairs in s-major order read each source row front
-// to back.
+// AlltoAll, native: unit = (pair p = s*n + r, unit of the chunk): chunk r of
+// rank s goes to chunk s of rank r.  Pairs in s-major order read each source
+// row front to back.
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
-a2a_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n) {
-    const size_t per = (m + kV<T> - 1) / kV<T>;
-    const size_t nn = static_cast<size_t>(n);
-    const size_t total = per * nn * nn;
-    const size_t T_ = threads_in_grid_x();
-    SegCursor cur(thread_in_grid_x(), T_, per);
-    for (size_t g = thread_in_grid_x(); g < total; g += kUnroll * T_) {
+a2a_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n,
+                  FastDiv per_chunk, FastDiv ranks) {
+    const uint32_t units = per_chunk.d * static_cast<uint32_t>(n) * static_cast<uint32_t>(n);
+    for_each_unit<kPc>(units, [&](uint32_t g) {
+        const uint32_t pair = fast_div(g, per_chunk);
+        const uint32_t s = fast_div(pair, ranks), r = pair - s * ranks.d;
+        const size_t unit = g - pair * per_chunk.d;
         RawVec<T, VEC> a[kUnroll];
         int valid[kUnroll];
-        T *dst[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const size_t s = cur.seg / nn, r = cur.seg - s * nn, j0 = cur.off * kV<T>;
-            valid[u] = g + u * T_ < total ? vec_valid<T>(cur.off, per, m) : 0;
-            dst[u] = recv + r * rstride + s * m + j0;
-            if (valid[u]) a[u].load(send + s * sstride + r * m + j0, valid[u]);
-            cur.next();
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u)
-            if (valid[u]) a[u].store(dst[u], valid[u]);
-    }
+        load_unit<T, VEC>(send + s * sstride + r * m, unit, m, a, valid);
+        store_unit<T, VEC>(recv + r * rstride + s * m, unit, a, valid);
+    });
 }
 
-// AlltoAll, FP8: unit = (pair, group of kJ blocks); blocks anchored at the
-// chunk start r*m.
+// AlltoAll, FP8: unit = (pair, kJ blocks); blocks anchored at the chunk start.
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
-a2a_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n) {
-    const size_t nbm = (m + kBlock - 1) / kBlock;
-    const size_t per = (nbm + kJ - 1) / kJ;
-    const size_t nn = static_cast<size_t>(n);
-    const size_t total = per * nn * nn;
+a2a_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n,
+               FastDiv per_chunk, FastDiv ranks) {
+    const uint32_t units = per_chunk.d * static_cast<uint32_t>(n) * static_cast<uint32_t>(n);
     const int e0 = lane_id() * 4;
-    SegCursor cur(warp_in_grid_x(), warps_in_grid_x(), per);
-    for (size_t g = warp_in_grid_x(); g < total; g += warps_in_grid_x(), cur.next()) {
-        const size_t s = cur.seg / nn, r = cur.seg - s * nn, b0 = cur.off * kJ;
-        const T *src = send + s * sstride + r * m;
-        T *dst = recv + r * rstride + s * m;
+    for_each_unit<kPg>(units, [&](uint32_t g) {
+        const uint32_t pair = fast_div(g, per_chunk);
+        const uint32_t s = fast_div(pair, ranks), r = pair - s * ranks.d;
+        const size_t b0 = static_cast<size_t>(g - pair * per_chunk.d) * kJ;
+        const T *src = send + static_cast<size_t>(s) * sstride + static_cast<size_t>(r) * m;
+        T *dst = recv + static_cast<size_t>(r) * rstride + static_cast<size_t>(s) * m;
         float v[kJ][4];
         int valid[kJ];
 #pragma unroll
@@ -262,7 +267,7 @@ a2a_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m,
         wire_fp8_blocks<kJ>(v);
 #pragma unroll
         for (int j = 0; j < kJ; ++j) store4<T, VEC>(dst + (b0 + j) * kBlock + e0, valid[j], v[j]);
-    }
+    });
 }
 
 // ------------------------------------------------------------- dispatching
@@ -275,25 +280,29 @@ cudaError_t dispatch(rlx_dtype dtype, bool vec, F &&f) {
 }
 
 template <typename K, typename... Args>
-cudaError_t launch(K kernel, unsigned segments, size_t jobs_per_segment, size_t jobs_per_cta,
-                   cudaStream_t stream, Args... args) {
-    const dim3 grid = grid_2d(reinterpret_cast<const void *>(kernel), segments,
-                              jobs_per_segment, jobs_per_cta);
+cudaError_t launch(K kernel, size_t units, size_t units_per_cta, cudaStream_t stream,
+                   Args... args) {
+    const dim3 grid = grid_for(reinterpret_cast<const void *>(kernel), units, units_per_cta);
+    if (grid.x == 0) return cudaErrorInvalidValue;
     kernel<<<grid, kThreads, 0, stream>>>(args...);
     return cudaGetLastError();
 }
 
 constexpr size_t kWarps = kThreads / 32;
 
-template <typename T> size_t nvec_of(size_t n) { return (n + kV<T> - 1) / kV<T>; }
-size_t nblk_of(size_t n) { return (n + kBlock - 1) / kBlock; }
+// units of kWarpVecs vectors, or of kJ / kJd blocks, in n elements
+template <typename T> size_t copy_units(size_t n) {
+    return ((n + kV<T> - 1) / kV<T> + kWarpVecs - 1) / kWarpVecs;
+}
+size_t block_units(size_t n, size_t per) { return ((n + kBlock - 1) / kBlock + per - 1) / per; }
+bool fits32(size_t v) { return v < (size_t{1} << 32); }
 
 }  // namespace
 
 cudaError_t launch_copy(const void *src, void *dst, size_t n, rlx_dtype dtype, bool vec,
                         cudaStream_t stream) {
     return dispatch(dtype, vec, [&]<typename T, bool VEC>() {
-        return launch(copy_kernel<T, VEC>, 1, nvec_of<T>(n), kThreads * kUnroll, stream,
+        return launch(copy_kernel<T, VEC>, copy_units<T>(n), kWarps * kPc, stream,
                       static_cast<const T *>(src), static_cast<T *>(dst), n);
     });
 }
@@ -304,12 +313,15 @@ cudaError_t launch_tree_gather(void *recv, size_t count, size_t stride, int nran
                                cudaStream_t stream) {
     return dispatch(dtype, vec, [&]<typename T, bool VEC>() {
         T *r = static_cast<T *>(recv);
-        if (wire == RLX_WIRE_NATIVE)
-            return launch(tree_gather_native_kernel<T, VEC>, 1,
-                          nvec_of<T>(chunk) * static_cast<size_t>(nranks), kThreads * kUnroll,
-                          stream, r, count, stride, nranks, chunk);
-        return launch(tree_gather_fp8_kernel<T, VEC>, 1, nblk_of(count), kWarps * kJd, stream, r,
-                      count, stride, nranks, ws_codes, ws_scales);
+        if (wire == RLX_WIRE_NATIVE) {
+            const size_t per = copy_units<T>(chunk);
+            if (!fits32(per)) return cudaErrorInvalidValue;
+            return launch(tree_gather_native_kernel<T, VEC>, per * static_cast<size_t>(nranks),
+                          kWarps * kPc, stream, r, count, stride, nranks, chunk,
+                          make_fastdiv(static_cast<uint32_t>(per)));
+        }
+        return launch(tree_gather_fp8_kernel<T, VEC>, block_units(count, kJd), kWarps * kPg,
+                      stream, r, count, stride, nranks, ws_codes, ws_scales);
     });
 }
 
@@ -320,11 +332,14 @@ cudaError_t launch_all_gather(const void *send, size_t send_stride, void *recv,
         const T *s = static_cast<const T *>(send);
         T *r = static_cast<T *>(recv);
         const size_t nn = static_cast<size_t>(nranks);
+        const size_t per = wire == RLX_WIRE_NATIVE ? copy_units<T>(m) : block_units(m, kJ);
+        if (!fits32(per)) return cudaErrorInvalidValue;
+        const FastDiv fd = make_fastdiv(static_cast<uint32_t>(per));
         if (wire == RLX_WIRE_NATIVE)
-            return launch(ag_native_kernel<T, VEC>, 1, nvec_of<T>(m) * nn, kThreads * kUnroll,
-                          stream, s, send_stride, r, recv_stride, m, nranks);
-        return launch(ag_fp8_kernel<T, VEC>, 1, nblk_of(m) * nn, kWarps * kJ, stream, s,
-                      send_stride, r, recv_stride, m, nranks);
+            return launch(ag_native_kernel<T, VEC>, per * nn, kWarps * kPc, stream, s,
+                          send_stride, r, recv_stride, m, nranks, fd);
+        return launch(ag_fp8_kernel<T, VEC>, per * nn, kWarps * kPg, stream, s, send_stride, r,
+                      recv_stride, m, nranks, fd);
     });
 }
 
@@ -335,11 +350,15 @@ cudaError_t launch_alltoall(const void *send, size_t send_stride, void *recv,
         const T *s = static_cast<const T *>(send);
         T *r = static_cast<T *>(recv);
         const size_t pairs = static_cast<size_t>(nranks) * static_cast<size_t>(nranks);
+        const size_t per = wire == RLX_WIRE_NATIVE ? copy_units<T>(m) : block_units(m, kJ);
+        if (!fits32(per)) return cudaErrorInvalidValue;
+        const FastDiv fd = make_fastdiv(static_cast<uint32_t>(per));
+        const FastDiv fn = make_fastdiv(static_cast<uint32_t>(nranks));
         if (wire == RLX_WIRE_NATIVE)
-            return launch(a2a_native_kernel<T, VEC>, 1, nvec_of<T>(m) * pairs, kThreads * kUnroll,
-                          stream, s, send_stride, r, recv_stride, m, nranks);
-        return launch(a2a_fp8_kernel<T, VEC>, 1, nblk_of(m) * pairs, kWarps * kJ, stream, s,
-                      send_stride, r, recv_stride, m, nranks);
+            return launch(a2a_native_kernel<T, VEC>, per * pairs, kWarps * kPc, stream, s,
+                          send_stride, r, recv_stride, m, nranks, fd, fn);
+        return launch(a2a_fp8_kernel<T, VEC>, per * pairs, kWarps * kPg, stream, s, send_stride,
+                      r, recv_stride, m, nranks, fd, fn);
     });
 }
 

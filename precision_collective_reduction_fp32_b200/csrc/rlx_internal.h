@@ -14,12 +14,11 @@ namespace rlx {
 
 constexpr int kThreads = 256;  // threads per CTA for every kernel
 
-// Grid for a persistent kernel over `segments` equal segments of work (grid
-// y) of `jobs_per_segment` units each, `jobs_per_cta` units per CTA and loop
-// iteration: x = enough CTAs for one segment, capped so that all segments
-// together use about (resident CTAs per SM) x (SM count) CTAs.
-dim3 grid_2d(const void *kernel, unsigned segments, size_t jobs_per_segment,
-             size_t jobs_per_cta);
+// Grid for `units` units of work, `units_per_cta` per CTA: one CTA per group
+// of units (the kernels loop if the grid is smaller).  The unit count must be
+// below 2^32 (the kernels index units with 32 bits); larger requests return
+// an empty grid.
+dim3 grid_for(const void *kernel, size_t units, size_t units_per_cta);
 
 // DDA-flat, all wires.  nranks >= 2.
 cudaError_t launch_allreduce_flat(const void *send, void *recv, size_t count, size_t stride,

@@ -6,102 +6,113 @@
 //
 // A warp handles kJ consecutive 128-element blocks of one row at once, 4
 // elements per lane per block: each block amax is one warp reduction, each
-// lane writes its 4 codes of a block as one 32-bit word.  Rows are the grid's
-// y dimension.
+// lane writes its 4 codes of a block as one 32-bit word.  Units (row, group
+// of kJ blocks) are numbered row-major and handed out in CTA-sized runs.
 #include "rlx_device.cuh"
 #include "rlx_internal.h"
 
 namespace rlx {
 namespace {
 
-constexpr int kJq = 4;   // blocks per warp, quantise
-constexpr int kJd = 8;   // blocks per warp, dequantise
+#ifndef RLX_JQ
+#define RLX_JQ 4
+#endif
+#ifndef RLX_JDQ
+#define RLX_JDQ 8
+#endif
+#ifndef RLX_P_Q
+#define RLX_P_Q 2
+#endif
+constexpr int kJq = RLX_JQ;    // blocks in flight per warp, quantise
+constexpr int kJd = RLX_JDQ;   // blocks in flight per warp, dequantise
+constexpr int kPq = RLX_P_Q;   // units per warp per CTA run
 
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 quantize_kernel(const T *x, size_t rows, size_t n, size_t stride, uint8_t *codes,
-                float *scales) {
+                float *scales, FastDiv per_row) {
     const size_t nbr = (n + kBlock - 1) / kBlock;
+    const uint32_t units = per_row.d * static_cast<uint32_t>(rows);
     const int e0 = lane_id() * 4;
-    for (size_t row = blockIdx.y; row < rows; row += gridDim.y) {
+    for_each_unit<kPq>(units, [&](uint32_t g) {
+        const uint32_t row = fast_div(g, per_row);
+        const size_t b0 = static_cast<size_t>(g - row * per_row.d) * kJq;
         const T *xr = x + row * stride;
         uint8_t *cr = codes + row * stride;
-        float *sr = scales + row * nbr;
-        for (size_t b0 = warp_in_grid_x() * kJq; b0 < nbr; b0 += warps_in_grid_x() * kJq) {
-            float v[kJq][4];
-            int valid[kJq];
-            float amax[kJq];
+        float v[kJq][4];
+        int valid[kJq];
+        float amax[kJq];
 #pragma unroll
-            for (int j = 0; j < kJq; ++j) {
-                valid[j] = lane_valid((b0 + j) * kBlock, n);
-                load4<T, VEC>(xr + (b0 + j) * kBlock + e0, valid[j], v[j]);
-            }
+        for (int j = 0; j < kJq; ++j) {
+            valid[j] = lane_valid((b0 + j) * kBlock, n);
+            load4<T, VEC>(xr + (b0 + j) * kBlock + e0, valid[j], v[j]);
+        }
 #pragma unroll
-            for (int j = 0; j < kJq; ++j) amax[j] = warp_amax4(v[j]);
-            Scale sc[kJq];
-            make_scales<kJq>(amax, sc);
+        for (int j = 0; j < kJq; ++j) amax[j] = warp_amax4(v[j]);
+        Scale sc[kJq];
+        make_scales<kJq>(amax, sc);
 #pragma unroll
-            for (int j = 0; j < kJq; ++j) {
-                const uint32_t q = quant4(v[j], sc[j]);
-                uint8_t *dst = cr + (b0 + j) * kBlock + e0;
-                if (VEC && valid[j] == 4) {
-                    __stcs(reinterpret_cast<unsigned int *>(dst), q);
-                } else {
+        for (int j = 0; j < kJq; ++j) {
+            const uint32_t q = quant4(v[j], sc[j]);
+            uint8_t *dst = cr + (b0 + j) * kBlock + e0;
+            if (VEC && valid[j] == 4) {
+                st_stream(reinterpret_cast<unsigned int *>(dst), q);
+            } else {
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        if (k < valid[j]) dst[k] = static_cast<uint8_t>(q >> (8 * k));
-                }
-            }
-            // lane j < kJq stores the scale of block b0 + j
-            const int l = lane_id();
-            if (l < kJq && b0 + l < nbr) {
-                float s = sc[0].s;
-#pragma unroll
-                for (int j = 1; j < kJq; ++j)
-                    if (l == j) s = sc[j].s;
-                __stcs(sr + b0 + l, s);
+                for (int k = 0; k < 4; ++k)
+                    if (k < valid[j]) dst[k] = static_cast<uint8_t>(q >> (8 * k));
             }
         }
-    }
+        // lane j < kJq stores the scale of block b0 + j
+        const int l = lane_id();
+        if (l < kJq && b0 + l < nbr) {
+            float s = sc[0].s;
+#pragma unroll
+            for (int j = 1; j < kJq; ++j)
+                if (l == j) s = sc[j].s;
+            st_stream(scales + row * nbr + b0 + l, s);
+        }
+    });
 }
 
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 dequantize_kernel(const uint8_t *codes, const float *scales, size_t rows, size_t n,
-                  size_t stride, T *y) {
+                  size_t stride, T *y, FastDiv per_row) {
     const size_t nbr = (n + kBlock - 1) / kBlock;
+    const uint32_t units = per_row.d * static_cast<uint32_t>(rows);
     const int e0 = lane_id() * 4;
-    for (size_t row = blockIdx.y; row < rows; row += gridDim.y) {
+    for_each_unit<kPq>(units, [&](uint32_t g) {
+        const uint32_t row = fast_div(g, per_row);
+        const size_t b0 = static_cast<size_t>(g - row * per_row.d) * kJd;
         const uint8_t *cr = codes + row * stride;
         const float *sr = scales + row * nbr;
         T *yr = y + row * stride;
-        for (size_t b0 = warp_in_grid_x() * kJd; b0 < nbr; b0 += warps_in_grid_x() * kJd) {
-            uint32_t q[kJd];
-            float s[kJd];
-            int valid[kJd];
+        uint32_t q[kJd];
+        float s[kJd];
+        int valid[kJd];
 #pragma unroll
-            for (int j = 0; j < kJd; ++j) {
-                const size_t b = b0 + j;
-                valid[j] = lane_valid(b * kBlock, n);
-                const uint8_t *src = cr + b * kBlock + e0;
-                q[j] = 0;
-                if (VEC && valid[j] == 4) {
-                    q[j] = __ldcs(reinterpret_cast<const unsigned int *>(src));
-                } else {
+        for (int j = 0; j < kJd; ++j) {
+            const size_t b = b0 + j;
+            valid[j] = lane_valid(b * kBlock, n);
+            const uint8_t *src = cr + b * kBlock + e0;
+            q[j] = 0;
+            if (VEC && valid[j] == 4) {
+                q[j] = ld_stream(reinterpret_cast<const unsigned int *>(src));
+            } else {
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        if (k < valid[j]) q[j] |= static_cast<uint32_t>(src[k]) << (8 * k);
-                }
-                s[j] = b < nbr ? __ldcs(sr + b) : 0.0f;
+                for (int k = 0; k < 4; ++k)
+                    if (k < valid[j]) q[j] |= static_cast<uint32_t>(src[k]) << (8 * k);
             }
-#pragma unroll
-            for (int j = 0; j < kJd; ++j) {
-                float v[4];
-                dequant4(q[j], s[j], v);
-                store4<T, VEC>(yr + (b0 + j) * kBlock + e0, valid[j], v);
-            }
+            s[j] = b < nbr ? ld_stream(sr + b) : 0.0f;
         }
-    }
+#pragma unroll
+        for (int j = 0; j < kJd; ++j) {
+            float v[4];
+            dequant4(q[j], s[j], v);
+            store4<T, VEC>(yr + (b0 + j) * kBlock + e0, valid[j], v);
+        }
+    });
 }
 
 template <typename F>
@@ -112,10 +123,16 @@ cudaError_t dispatch(rlx_dtype dtype, bool vec, F &&f) {
 }
 
 constexpr size_t kWarps = kThreads / 32;
-constexpr unsigned kMaxGridY = 65535;
 
-unsigned row_segments(size_t rows) {
-    return rows < kMaxGridY ? static_cast<unsigned>(rows) : kMaxGridY;
+template <typename K, typename... Args>
+cudaError_t launch_rows(K kernel, size_t rows, size_t n, size_t blocks_per_unit,
+                        cudaStream_t stream, Args... args) {
+    const size_t per = ((n + kBlock - 1) / kBlock + blocks_per_unit - 1) / blocks_per_unit;
+    if (per >= (size_t{1} << 32) || rows >= (size_t{1} << 32)) return cudaErrorInvalidValue;
+    const dim3 grid = grid_for(reinterpret_cast<const void *>(kernel), per * rows, kWarps * kPq);
+    if (grid.x == 0) return cudaErrorInvalidValue;
+    kernel<<<grid, kThreads, 0, stream>>>(args..., make_fastdiv(static_cast<uint32_t>(per)));
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -124,11 +141,8 @@ cudaError_t launch_quantize(const void *x, rlx_dtype dtype, size_t rows, size_t 
                             size_t stride, uint8_t *codes, float *scales, bool vec,
                             cudaStream_t stream) {
     return dispatch(dtype, vec, [&]<typename T, bool VEC>() {
-        auto k = quantize_kernel<T, VEC>;
-        const dim3 grid = grid_2d(reinterpret_cast<const void *>(k), row_segments(rows),
-                                  (n + kBlock - 1) / kBlock, kWarps * kJq);
-        k<<<grid, kThreads, 0, stream>>>(static_cast<const T *>(x), rows, n, stride, codes, scales);
-        return cudaGetLastError();
+        return launch_rows(quantize_kernel<T, VEC>, rows, n, kJq, stream,
+                           static_cast<const T *>(x), rows, n, stride, codes, scales);
     });
 }
 
@@ -136,11 +150,8 @@ cudaError_t launch_dequantize(const uint8_t *codes, const float *scales, size_t 
                               size_t n, size_t stride, void *y, rlx_dtype dtype, bool vec,
                               cudaStream_t stream) {
     return dispatch(dtype, vec, [&]<typename T, bool VEC>() {
-        auto k = dequantize_kernel<T, VEC>;
-        const dim3 grid = grid_2d(reinterpret_cast<const void *>(k), row_segments(rows),
-                                  (n + kBlock - 1) / kBlock, kWarps * kJd);
-        k<<<grid, kThreads, 0, stream>>>(codes, scales, rows, n, stride, static_cast<T *>(y));
-        return cudaGetLastError();
+        return launch_rows(dequantize_kernel<T, VEC>, rows, n, kJd, stream, codes, scales, rows,
+                           n, stride, static_cast<T *>(y));
     });
 }
 

@@ -17,9 +17,9 @@
 //   FP8 wire: one warp per 128-element block, 4 elements per lane, so a block
 //     amax is one warp reduction; the warp loads the block from all N ranks,
 //     dequantises each rank's quantised block and sums in rank order.
-// Chunked passes walk (chunk, unit) segment-major with a SegCursor: all warps
-// stay within about one chunk, which keeps few DRAM streams open, and no
-// index is divided per step.
+// Units of work are numbered in memory order (chunk-major for chunked
+// passes) and handed out in CTA-sized runs by for_each_unit, so the CTAs in
+// flight stream one compact stretch of every row.
 #include "rlx_device.cuh"
 #include "rlx_internal.h"
 
@@ -35,7 +35,7 @@ template <typename T, bool VEC>
 __device__ __forceinline__ void loadv(const T *p, int valid, float (&v)[VecN<T>::n]) {
     constexpr int V = VecN<T>::n;
     if (VEC && valid == V) {
-        const uint4 q = __ldcs(reinterpret_cast<const uint4 *>(p));
+        const uint4 q = ld_stream(reinterpret_cast<const uint4 *>(p));
         if constexpr (sizeof(T) == 4) {
             v[0] = __uint_as_float(q.x); v[1] = __uint_as_float(q.y);
             v[2] = __uint_as_float(q.z); v[3] = __uint_as_float(q.w);
@@ -69,7 +69,7 @@ __device__ __forceinline__ void storev(T *p, int valid, const float (&v)[VecN<T>
                        (static_cast<uint32_t>(f32_to_bf16_bits(v[2 * k + 1])) << 16);
             q = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        __stcs(reinterpret_cast<uint4 *>(p), q);
+        st_stream(reinterpret_cast<uint4 *>(p), q);
     } else {
 #pragma unroll
         for (int k = 0; k < V; ++k)
@@ -128,65 +128,81 @@ __device__ __forceinline__ void reduce_block_fp8(const T *src, size_t pitch, int
 
 // ------------------------------------------------------------------ kernels
 
+// Units per warp (per CTA run) of each kernel.
+#ifndef RLX_P_NATIVE
+#define RLX_P_NATIVE 1
+#endif
+#ifndef RLX_P_FP8
+#define RLX_P_FP8 4
+#endif
+constexpr int kPn = RLX_P_NATIVE;
+constexpr int kPf = RLX_P_FP8;
+
+// DDA-flat, native: unit g = 32 consecutive 16-byte vectors (lane l: 32g + l).
 template <typename T, int NR, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 flat_native_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
     constexpr int V = VecN<T>::n;
     const size_t nvec = (count + V - 1) / V;
-    for (size_t v = thread_in_grid_x(); v < nvec; v += threads_in_grid_x()) {
+    const uint32_t units = static_cast<uint32_t>((nvec + 31) / 32);
+    for_each_unit<kPn>(units, [&](uint32_t g) {
+        const size_t v = static_cast<size_t>(g) * 32 + lane_id();
+        if (v >= nvec) return;
         const size_t i0 = v * V;
         const int valid = count - i0 < static_cast<size_t>(V) ? static_cast<int>(count - i0) : V;
         float acc[V];
         reduce_vec<T, NR, VEC>(send + i0, stride, n, valid, acc);
         for (int r = 0; r < n; ++r) storev<T, VEC>(recv + r * stride + i0, valid, acc);
-    }
+    });
 }
 
+// DDA-flat, FP8: unit g = 128-block g.
 template <typename T, int NR, bool VEC>
 __global__ void __launch_bounds__(kThreads, NR <= 8 ? 3 : 1)
 flat_fp8_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
-    const size_t nblk = (count + kBlock - 1) / kBlock;
+    const uint32_t nblk = static_cast<uint32_t>((count + kBlock - 1) / kBlock);
     const int e0 = lane_id() * 4;
-    for (size_t b = warp_in_grid_x(); b < nblk; b += warps_in_grid_x()) {
-        const size_t base = b * kBlock;
+    for_each_unit<kPf>(nblk, [&](uint32_t b) {
+        const size_t base = static_cast<size_t>(b) * kBlock;
         const int valid = lane_valid(base, count);
         float acc[4];
         reduce_block_fp8<T, NR, VEC>(send + base, stride, n, valid, acc);
         for (int r = 0; r < n; ++r) store4<T, VEC>(recv + r * stride + base + e0, valid, acc);
-    }
+    });
 }
 
-// DDA-tree pass 1, native: chunk c -> row c of recv.
+// DDA-tree pass 1, native: unit = (chunk c, 32 vectors of it); chunk c -> row c.
 template <typename T, int NR, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 tree_reduce_native_kernel(const T *send, T *recv, size_t count, size_t stride, int n,
-                          size_t chunk) {
+                          size_t chunk, FastDiv per_chunk) {
     constexpr int V = VecN<T>::n;
-    const size_t per = (chunk + V - 1) / V;
-    const size_t total = per * static_cast<size_t>(n);
-    SegCursor cur(thread_in_grid_x(), threads_in_grid_x(), per);
-    for (size_t g = thread_in_grid_x(); g < total; g += threads_in_grid_x(), cur.next()) {
-        const size_t lo = cur.seg * chunk;
-        const size_t i0 = lo + cur.off * V;
-        if (i0 >= count) continue;
+    const uint32_t units = per_chunk.d * static_cast<uint32_t>(n);
+    for_each_unit<kPn>(units, [&](uint32_t g) {
+        const uint32_t c = fast_div(g, per_chunk);
+        const size_t lo = static_cast<size_t>(c) * chunk;
+        if (lo >= count) return;
+        const size_t i0 = lo + (static_cast<size_t>(g - c * per_chunk.d) * 32 + lane_id()) * V;
         const size_t hi = count - lo < chunk ? count : lo + chunk;
+        if (i0 >= hi) return;
         const int valid = hi - i0 < static_cast<size_t>(V) ? static_cast<int>(hi - i0) : V;
         float acc[V];
         reduce_vec<T, NR, VEC>(send + i0, stride, n, valid, acc);
-        storev<T, VEC>(recv + cur.seg * stride + i0, valid, acc);
-    }
+        storev<T, VEC>(recv + c * stride + i0, valid, acc);
+    });
 }
 
-// DDA-tree pass 1, FP8: reduce, then quantise the reduced block again into
-// the workspace payload (codes padded to whole blocks, one scale per block).
+// DDA-tree pass 1, FP8: unit = 128-block; reduce, then quantise the reduced
+// block again into the workspace payload (codes padded to whole blocks, one
+// scale per block).
 template <typename T, int NR, bool VEC>
 __global__ void __launch_bounds__(kThreads, NR <= 8 ? 3 : 1)
 tree_reduce_fp8_kernel(const T *send, size_t count, size_t stride, int n,
                        uint8_t *ws_codes, float *ws_scales) {
-    const size_t nblk = (count + kBlock - 1) / kBlock;
+    const uint32_t nblk = static_cast<uint32_t>((count + kBlock - 1) / kBlock);
     const int e0 = lane_id() * 4;
-    for (size_t b = warp_in_grid_x(); b < nblk; b += warps_in_grid_x()) {
-        const size_t base = b * kBlock;
+    for_each_unit<kPf>(nblk, [&](uint32_t b) {
+        const size_t base = static_cast<size_t>(b) * kBlock;
         float acc[4];
         reduce_block_fp8<T, NR, VEC>(send + base, stride, n, lane_valid(base, count), acc);
         const Scale sc = make_scale(warp_amax4(acc));
@@ -194,42 +210,43 @@ tree_reduce_fp8_kernel(const T *send, size_t count, size_t stride, int n,
         // default caching: pass 2 reads the payload back right away
         *reinterpret_cast<uint32_t *>(ws_codes + base + e0) = codes;
         if (lane_id() == 0) ws_scales[b] = sc.s;
-    }
+    });
 }
 
-// ReduceScatter, native: unit = (destination rank r, vector of chunk r).
+// ReduceScatter, native: unit = (destination rank r, 32 vectors of chunk r).
 template <typename T, int NR, bool VEC>
 __global__ void __launch_bounds__(kThreads)
-rs_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n) {
+rs_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n,
+                 FastDiv per_chunk) {
     constexpr int V = VecN<T>::n;
-    const size_t per = (m + V - 1) / V;
-    const size_t total = per * static_cast<size_t>(n);
-    SegCursor cur(thread_in_grid_x(), threads_in_grid_x(), per);
-    for (size_t g = thread_in_grid_x(); g < total; g += threads_in_grid_x(), cur.next()) {
-        const size_t r = cur.seg, j0 = cur.off * V;
+    const uint32_t units = per_chunk.d * static_cast<uint32_t>(n);
+    for_each_unit<kPn>(units, [&](uint32_t g) {
+        const uint32_t r = fast_div(g, per_chunk);
+        const size_t j0 = (static_cast<size_t>(g - r * per_chunk.d) * 32 + lane_id()) * V;
+        if (j0 >= m) return;
         const int valid = m - j0 < static_cast<size_t>(V) ? static_cast<int>(m - j0) : V;
         float acc[V];
         reduce_vec<T, NR, VEC>(send + r * m + j0, sstride, n, valid, acc);
         storev<T, VEC>(recv + r * rstride + j0, valid, acc);
-    }
+    });
 }
 
 // ReduceScatter, FP8: unit = (destination rank r, 128-block of chunk r);
 // blocks anchored at the chunk start r*m.
 template <typename T, int NR, bool VEC>
 __global__ void __launch_bounds__(kThreads, NR <= 8 ? 3 : 1)
-rs_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n) {
-    const size_t per = (m + kBlock - 1) / kBlock;
-    const size_t total = per * static_cast<size_t>(n);
+rs_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n,
+              FastDiv per_chunk) {
+    const uint32_t units = per_chunk.d * static_cast<uint32_t>(n);
     const int e0 = lane_id() * 4;
-    SegCursor cur(warp_in_grid_x(), warps_in_grid_x(), per);
-    for (size_t g = warp_in_grid_x(); g < total; g += warps_in_grid_x(), cur.next()) {
-        const size_t r = cur.seg, j0 = cur.off * kBlock;
+    for_each_unit<kPf>(units, [&](uint32_t g) {
+        const uint32_t r = fast_div(g, per_chunk);
+        const size_t j0 = static_cast<size_t>(g - r * per_chunk.d) * kBlock;
         const int valid = lane_valid(j0, m);
         float acc[4];
         reduce_block_fp8<T, NR, VEC>(send + r * m + j0, sstride, n, valid, acc);
         store4<T, VEC>(recv + r * rstride + j0 + e0, valid, acc);
-    }
+    });
 }
 
 // ------------------------------------------------------------- dispatching
@@ -250,10 +267,10 @@ cudaError_t dispatch(rlx_dtype dtype, int n, bool vec, F &&f) {
 }
 
 template <typename K, typename... Args>
-cudaError_t launch(K kernel, unsigned segments, size_t jobs_per_segment, size_t jobs_per_cta,
-                   cudaStream_t stream, Args... args) {
-    const dim3 grid = grid_2d(reinterpret_cast<const void *>(kernel), segments,
-                              jobs_per_segment, jobs_per_cta);
+cudaError_t launch(K kernel, size_t units, size_t units_per_cta, cudaStream_t stream,
+                   Args... args) {
+    const dim3 grid = grid_for(reinterpret_cast<const void *>(kernel), units, units_per_cta);
+    if (grid.x == 0) return cudaErrorInvalidValue;
     kernel<<<grid, kThreads, 0, stream>>>(args...);
     return cudaGetLastError();
 }
@@ -269,13 +286,13 @@ cudaError_t launch_allreduce_flat(const void *send, void *recv, size_t count, si
         const T *s = static_cast<const T *>(send);
         T *r = static_cast<T *>(recv);
         if (wire == RLX_WIRE_NATIVE) {
-            const size_t nvec = (count + VecN<T>::n - 1) / VecN<T>::n;
-            return launch(flat_native_kernel<T, NR, VEC>, 1, nvec, kThreads, stream, s, r, count,
-                          stride, nranks);
+            const size_t units = ((count + VecN<T>::n - 1) / VecN<T>::n + 31) / 32;
+            return launch(flat_native_kernel<T, NR, VEC>, units, kWarps * kPn, stream, s, r,
+                          count, stride, nranks);
         }
         const size_t nblk = (count + kBlock - 1) / kBlock;
-        return launch(flat_fp8_kernel<T, NR, VEC>, 1, nblk, kWarps, stream, s, r, count, stride,
-                      nranks);
+        return launch(flat_fp8_kernel<T, NR, VEC>, nblk, kWarps * kPf, stream, s, r, count,
+                      stride, nranks);
     });
 }
 
@@ -286,13 +303,15 @@ cudaError_t launch_tree_reduce(const void *send, void *recv, size_t count, size_
     return dispatch(dtype, nranks, vec, [&]<typename T, int NR, bool VEC>() {
         const T *s = static_cast<const T *>(send);
         if (wire == RLX_WIRE_NATIVE) {
-            const size_t nvec = (chunk + VecN<T>::n - 1) / VecN<T>::n;
-            return launch(tree_reduce_native_kernel<T, NR, VEC>, 1,
-                          nvec * static_cast<size_t>(nranks), kThreads, stream, s,
-                          static_cast<T *>(recv), count, stride, nranks, chunk);
+            const size_t per = ((chunk + VecN<T>::n - 1) / VecN<T>::n + 31) / 32;
+            if (per >= (size_t{1} << 32)) return cudaErrorInvalidValue;
+            return launch(tree_reduce_native_kernel<T, NR, VEC>,
+                          per * static_cast<size_t>(nranks), kWarps * kPn, stream, s,
+                          static_cast<T *>(recv), count, stride, nranks, chunk,
+                          make_fastdiv(static_cast<uint32_t>(per)));
         }
         const size_t nblk = (count + kBlock - 1) / kBlock;
-        return launch(tree_reduce_fp8_kernel<T, NR, VEC>, 1, nblk, kWarps, stream, s, count,
+        return launch(tree_reduce_fp8_kernel<T, NR, VEC>, nblk, kWarps * kPf, stream, s, count,
                       stride, nranks, ws_codes, ws_scales);
     });
 }
@@ -304,14 +323,15 @@ cudaError_t launch_reduce_scatter(const void *send, size_t send_stride, void *re
         const T *s = static_cast<const T *>(send);
         T *r = static_cast<T *>(recv);
         const size_t nn = static_cast<size_t>(nranks);
-        if (wire == RLX_WIRE_NATIVE) {
-            const size_t nvec = (m + VecN<T>::n - 1) / VecN<T>::n;
-            return launch(rs_native_kernel<T, NR, VEC>, 1, nvec * nn, kThreads, stream, s,
-                          send_stride, r, recv_stride, m, nranks);
-        }
-        const size_t nbm = (m + kBlock - 1) / kBlock;
-        return launch(rs_fp8_kernel<T, NR, VEC>, 1, nbm * nn, kWarps, stream, s, send_stride, r,
-                      recv_stride, m, nranks);
+        const size_t per = wire == RLX_WIRE_NATIVE ? ((m + VecN<T>::n - 1) / VecN<T>::n + 31) / 32
+                                                   : (m + kBlock - 1) / kBlock;
+        if (per >= (size_t{1} << 32)) return cudaErrorInvalidValue;
+        const FastDiv fd = make_fastdiv(static_cast<uint32_t>(per));
+        if (wire == RLX_WIRE_NATIVE)
+            return launch(rs_native_kernel<T, NR, VEC>, per * nn, kWarps * kPn, stream, s,
+                          send_stride, r, recv_stride, m, nranks, fd);
+        return launch(rs_fp8_kernel<T, NR, VEC>, per * nn, kWarps * kPf, stream, s, send_stride,
+                      r, recv_stride, m, nranks, fd);
     });
 }
 
