@@ -21,11 +21,15 @@ namespace {
 #define RLX_JDQ 8
 #endif
 #ifndef RLX_P_Q
-#define RLX_P_Q 2
+#define RLX_P_Q 4
+#endif
+#ifndef RLX_P_DQ
+#define RLX_P_DQ 1
 #endif
 constexpr int kJq = RLX_JQ;    // blocks in flight per warp, quantise
 constexpr int kJd = RLX_JDQ;   // blocks in flight per warp, dequantise
-constexpr int kPq = RLX_P_Q;   // units per warp per CTA run
+constexpr int kPq = RLX_P_Q;   // units per warp per CTA run, quantise
+constexpr int kPdq = RLX_P_DQ; // units per warp per CTA run, dequantise
 
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
@@ -82,7 +86,7 @@ dequantize_kernel(const uint8_t *codes, const float *scales, size_t rows, size_t
     const size_t nbr = (n + kBlock - 1) / kBlock;
     const uint32_t units = per_row.d * static_cast<uint32_t>(rows);
     const int e0 = lane_id() * 4;
-    for_each_unit<kPq>(units, [&](uint32_t g) {
+    for_each_unit<kPdq>(units, [&](uint32_t g) {
         const uint32_t row = fast_div(g, per_row);
         const size_t b0 = static_cast<size_t>(g - row * per_row.d) * kJd;
         const uint8_t *cr = codes + row * stride;
@@ -126,10 +130,11 @@ constexpr size_t kWarps = kThreads / 32;
 
 template <typename K, typename... Args>
 cudaError_t launch_rows(K kernel, size_t rows, size_t n, size_t blocks_per_unit,
-                        cudaStream_t stream, Args... args) {
+                        size_t units_per_warp, cudaStream_t stream, Args... args) {
     const size_t per = ((n + kBlock - 1) / kBlock + blocks_per_unit - 1) / blocks_per_unit;
     if (per >= (size_t{1} << 32) || rows >= (size_t{1} << 32)) return cudaErrorInvalidValue;
-    const dim3 grid = grid_for(reinterpret_cast<const void *>(kernel), per * rows, kWarps * kPq);
+    const dim3 grid = grid_for(reinterpret_cast<const void *>(kernel), per * rows,
+                               kWarps * units_per_warp);
     if (grid.x == 0) return cudaErrorInvalidValue;
     kernel<<<grid, kThreads, 0, stream>>>(args..., make_fastdiv(static_cast<uint32_t>(per)));
     return cudaGetLastError();
@@ -141,7 +146,7 @@ cudaError_t launch_quantize(const void *x, rlx_dtype dtype, size_t rows, size_t 
                             size_t stride, uint8_t *codes, float *scales, bool vec,
                             cudaStream_t stream) {
     return dispatch(dtype, vec, [&]<typename T, bool VEC>() {
-        return launch_rows(quantize_kernel<T, VEC>, rows, n, kJq, stream,
+        return launch_rows(quantize_kernel<T, VEC>, rows, n, kJq, kPq, stream,
                            static_cast<const T *>(x), rows, n, stride, codes, scales);
     });
 }
@@ -150,7 +155,7 @@ cudaError_t launch_dequantize(const uint8_t *codes, const float *scales, size_t 
                               size_t n, size_t stride, void *y, rlx_dtype dtype, bool vec,
                               cudaStream_t stream) {
     return dispatch(dtype, vec, [&]<typename T, bool VEC>() {
-        return launch_rows(dequantize_kernel<T, VEC>, rows, n, kJd, stream, codes, scales, rows,
+        return launch_rows(dequantize_kernel<T, VEC>, rows, n, kJd, kPdq, stream, codes, scales, rows,
                            n, stride, static_cast<T *>(y));
     });
 }

@@ -133,7 +133,7 @@ __device__ __forceinline__ void reduce_block_fp8(const T *src, size_t pitch, int
 #define RLX_P_NATIVE 1
 #endif
 #ifndef RLX_P_FP8
-#define RLX_P_FP8 4
+#define RLX_P_FP8 2
 #endif
 constexpr int kPn = RLX_P_NATIVE;
 constexpr int kPf = RLX_P_FP8;
