@@ -10,6 +10,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <type_traits>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -293,6 +294,16 @@ __device__ __forceinline__ void for_each_unit(uint32_t total, F &&f) {
             if (g < total) f(static_cast<uint32_t>(g));
         }
     }
+}
+
+// Calls f(std::true_type{}) when the unit lies wholly inside its segment
+// (every lane owns a full vector of every block), else f(std::false_type{}).
+// The two instantiations let the compiler drop all bounds checks, and fold
+// the block offsets into the load and store instructions, on full units.
+template <typename F>
+__device__ __forceinline__ void with_full(bool full, F &&f) {
+    if (full) f(std::true_type{});
+    else f(std::false_type{});
 }
 
 // Elements of a 128-block that belong to this lane: 0..4.

@@ -95,18 +95,20 @@ __device__ __forceinline__ int vec_valid(size_t v, size_t nvec, size_t len) {
 // each warp store continues the previous one.
 constexpr int kWarpVecs = 32 * kUnroll;
 
-// Loads the unit's vectors of a segment of `len` elements at `src`.
-template <typename T, bool VEC, bool CACHED = false>
-__device__ __forceinline__ void load_unit(const T *src, size_t unit, size_t len,
+// Loads the unit's vectors of a segment of `len` elements at `src` (Full:
+// the unit lies wholly inside the segment, no bounds checks).
+template <typename T, bool VEC, bool CACHED = false, typename Full>
+__device__ __forceinline__ void load_unit(const T *src, size_t unit, size_t len, Full,
                                           RawVec<T, VEC> (&a)[kUnroll], int (&valid)[kUnroll]) {
     const size_t nv = (len + kV<T> - 1) / kV<T>;
+    const T *p = src + (unit * kWarpVecs + lane_id()) * kV<T>;
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-        const size_t v = unit * kWarpVecs + u * 32 + lane_id();
-        valid[u] = vec_valid<T>(v, nv, len);
+        if constexpr (Full::value) valid[u] = kV<T>;
+        else valid[u] = vec_valid<T>(unit * kWarpVecs + u * 32 + lane_id(), nv, len);
         if (valid[u]) {
-            if (CACHED) a[u].load_cached(src + v * kV<T>, valid[u]);
-            else a[u].load(src + v * kV<T>, valid[u]);
+            if (CACHED) a[u].load_cached(p + u * 32 * kV<T>, valid[u]);
+            else a[u].load(p + u * 32 * kV<T>, valid[u]);
         }
     }
 }
@@ -114,9 +116,16 @@ __device__ __forceinline__ void load_unit(const T *src, size_t unit, size_t len,
 template <typename T, bool VEC>
 __device__ __forceinline__ void store_unit(T *dst, size_t unit, const RawVec<T, VEC> (&a)[kUnroll],
                                            const int (&valid)[kUnroll]) {
+    T *p = dst + (unit * kWarpVecs + lane_id()) * kV<T>;
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u)
-        if (valid[u]) a[u].store(dst + (unit * kWarpVecs + u * 32 + lane_id()) * kV<T>, valid[u]);
+        if (valid[u]) a[u].store(p + u * 32 * kV<T>, valid[u]);
+}
+
+// Is unit `unit` (of kWarpVecs vectors) wholly inside a segment of len elements?
+template <typename T>
+__device__ __forceinline__ bool unit_full(size_t unit, size_t len) {
+    return (unit + 1) * kWarpVecs * kV<T> <= len;
 }
 
 template <typename T, bool VEC>
@@ -124,10 +133,12 @@ __global__ void __launch_bounds__(kThreads)
 copy_kernel(const T *src, T *dst, size_t n) {
     const uint32_t units = static_cast<uint32_t>(((n + kV<T> - 1) / kV<T> + kWarpVecs - 1) / kWarpVecs);
     for_each_unit<kPc>(units, [&](uint32_t g) {
-        RawVec<T, VEC> a[kUnroll];
-        int valid[kUnroll];
-        load_unit<T, VEC>(src, g, n, a, valid);
-        store_unit<T, VEC>(dst, g, a, valid);
+        with_full(unit_full<T>(g, n), [&](auto full) {
+            RawVec<T, VEC> a[kUnroll];
+            int valid[kUnroll];
+            load_unit<T, VEC>(src, g, n, full, a, valid);
+            store_unit<T, VEC>(dst, g, a, valid);
+        });
     });
 }
 
@@ -144,12 +155,15 @@ tree_gather_native_kernel(T *recv, size_t count, size_t stride, int n, size_t ch
         if (lo >= count) return;
         const size_t len = count - lo < chunk ? count - lo : chunk;
         const size_t unit = g - c * per_chunk.d;
-        RawVec<T, VEC> a[kUnroll];
-        int valid[kUnroll];
-        // the owner's chunk was just written by pass 1: default caching
-        load_unit<T, VEC, true>(recv + c * stride + lo, unit, len, a, valid);
-        for (int r = 0; r < n; ++r)
-            if (static_cast<uint32_t>(r) != c) store_unit<T, VEC>(recv + r * stride + lo, unit, a, valid);
+        with_full(unit_full<T>(unit, len), [&](auto full) {
+            RawVec<T, VEC> a[kUnroll];
+            int valid[kUnroll];
+            // the owner's chunk was just written by pass 1: default caching
+            load_unit<T, VEC, true>(recv + c * stride + lo, unit, len, full, a, valid);
+            for (int r = 0; r < n; ++r)
+                if (static_cast<uint32_t>(r) != c)
+                    store_unit<T, VEC>(recv + r * stride + lo, unit, a, valid);
+        });
     });
 }
 
@@ -163,21 +177,26 @@ tree_gather_fp8_kernel(T *recv, size_t count, size_t stride, int n, const uint8_
     const int e0 = lane_id() * 4;
     for_each_unit<kPg>(units, [&](uint32_t g) {
         const size_t b0 = static_cast<size_t>(g) * kJd;
-        float y[kJd][4];
-        int valid[kJd];
+        with_full((b0 + kJd) * kBlock <= count, [&](auto full) {
+            constexpr bool F = decltype(full)::value;
+            const uint8_t *cp = ws_codes + b0 * kBlock + e0;
+            float y[kJd][4];
+            int valid[kJd];
 #pragma unroll
-        for (int j = 0; j < kJd; ++j) {
-            const size_t b = b0 + j;
-            valid[j] = lane_valid(b * kBlock, count);
-            if (b < nblk) {
-                const uint32_t codes = *reinterpret_cast<const uint32_t *>(ws_codes + b * kBlock + e0);
-                dequant4(codes, ws_scales[b], y[j]);
+            for (int j = 0; j < kJd; ++j) {
+                const size_t b = b0 + j;
+                valid[j] = F ? 4 : lane_valid(b * kBlock, count);
+                if (F || b < nblk) {
+                    const uint32_t codes = *reinterpret_cast<const uint32_t *>(cp + j * kBlock);
+                    dequant4(codes, ws_scales[b], y[j]);
+                }
             }
-        }
-        for (int r = 0; r < n; ++r)
+            for (int r = 0; r < n; ++r) {
+                T *dst = recv + r * stride + b0 * kBlock + e0;
 #pragma unroll
-            for (int j = 0; j < kJd; ++j)
-                store4<T, VEC>(recv + r * stride + (b0 + j) * kBlock + e0, valid[j], y[j]);
+                for (int j = 0; j < kJd; ++j) store4<T, VEC>(dst + j * kBlock, valid[j], y[j]);
+            }
+        });
     });
 }
 
@@ -190,10 +209,12 @@ ag_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t 
     for_each_unit<kPc>(units, [&](uint32_t g) {
         const uint32_t s = fast_div(g, per_row);
         const size_t unit = g - s * per_row.d;
-        RawVec<T, VEC> a[kUnroll];
-        int valid[kUnroll];
-        load_unit<T, VEC>(send + s * sstride, unit, m, a, valid);
-        for (int r = 0; r < n; ++r) store_unit<T, VEC>(recv + r * rstride + s * m, unit, a, valid);
+        with_full(unit_full<T>(unit, m), [&](auto full) {
+            RawVec<T, VEC> a[kUnroll];
+            int valid[kUnroll];
+            load_unit<T, VEC>(send + s * sstride, unit, m, full, a, valid);
+            for (int r = 0; r < n; ++r) store_unit<T, VEC>(recv + r * rstride + s * m, unit, a, valid);
+        });
     });
 }
 
@@ -208,20 +229,22 @@ ag_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, 
     for_each_unit<kPg>(units, [&](uint32_t g) {
         const uint32_t s = fast_div(g, per_row);
         const size_t b0 = static_cast<size_t>(g - s * per_row.d) * kJ;
-        const T *src = send + s * sstride;
-        float v[kJ][4];
-        int valid[kJ];
+        with_full((b0 + kJ) * kBlock <= m, [&](auto full) {
+            const T *src = send + s * sstride + b0 * kBlock + e0;
+            float v[kJ][4];
+            int valid[kJ];
 #pragma unroll
-        for (int j = 0; j < kJ; ++j) {
-            valid[j] = lane_valid((b0 + j) * kBlock, m);
-            load4<T, VEC>(src + (b0 + j) * kBlock + e0, valid[j], v[j]);
-        }
-        wire_fp8_blocks<kJ>(v);
-        for (int r = 0; r < n; ++r) {
-            T *dst = recv + r * rstride + s * m;
+            for (int j = 0; j < kJ; ++j) {
+                valid[j] = decltype(full)::value ? 4 : lane_valid((b0 + j) * kBlock, m);
+                load4<T, VEC>(src + j * kBlock, valid[j], v[j]);
+            }
+            wire_fp8_blocks<kJ>(v);
+            for (int r = 0; r < n; ++r) {
+                T *dst = recv + r * rstride + s * m + b0 * kBlock + e0;
 #pragma unroll
-            for (int j = 0; j < kJ; ++j) store4<T, VEC>(dst + (b0 + j) * kBlock + e0, valid[j], v[j]);
-        }
+                for (int j = 0; j < kJ; ++j) store4<T, VEC>(dst + j * kBlock, valid[j], v[j]);
+            }
+        });
     });
 }
 
@@ -237,10 +260,14 @@ a2a_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t
         const uint32_t pair = fast_div(g, per_chunk);
         const uint32_t s = fast_div(pair, ranks), r = pair - s * ranks.d;
         const size_t unit = g - pair * per_chunk.d;
-        RawVec<T, VEC> a[kUnroll];
-        int valid[kUnroll];
-        load_unit<T, VEC>(send + s * sstride + r * m, unit, m, a, valid);
-        store_unit<T, VEC>(recv + r * rstride + s * m, unit, a, valid);
+        with_full(unit_full<T>(unit, m), [&](auto full) {
+            RawVec<T, VEC> a[kUnroll];
+            int valid[kUnroll];
+            load_unit<T, VEC>(send + static_cast<size_t>(s) * sstride + static_cast<size_t>(r) * m,
+                              unit, m, full, a, valid);
+            store_unit<T, VEC>(recv + static_cast<size_t>(r) * rstride + static_cast<size_t>(s) * m,
+                               unit, a, valid);
+        });
     });
 }
 
@@ -255,18 +282,22 @@ a2a_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m,
         const uint32_t pair = fast_div(g, per_chunk);
         const uint32_t s = fast_div(pair, ranks), r = pair - s * ranks.d;
         const size_t b0 = static_cast<size_t>(g - pair * per_chunk.d) * kJ;
-        const T *src = send + static_cast<size_t>(s) * sstride + static_cast<size_t>(r) * m;
-        T *dst = recv + static_cast<size_t>(r) * rstride + static_cast<size_t>(s) * m;
-        float v[kJ][4];
-        int valid[kJ];
+        with_full((b0 + kJ) * kBlock <= m, [&](auto full) {
+            const T *src = send + static_cast<size_t>(s) * sstride + static_cast<size_t>(r) * m +
+                           b0 * kBlock + e0;
+            T *dst = recv + static_cast<size_t>(r) * rstride + static_cast<size_t>(s) * m +
+                     b0 * kBlock + e0;
+            float v[kJ][4];
+            int valid[kJ];
 #pragma unroll
-        for (int j = 0; j < kJ; ++j) {
-            valid[j] = lane_valid((b0 + j) * kBlock, m);
-            load4<T, VEC>(src + (b0 + j) * kBlock + e0, valid[j], v[j]);
-        }
-        wire_fp8_blocks<kJ>(v);
+            for (int j = 0; j < kJ; ++j) {
+                valid[j] = decltype(full)::value ? 4 : lane_valid((b0 + j) * kBlock, m);
+                load4<T, VEC>(src + j * kBlock, valid[j], v[j]);
+            }
+            wire_fp8_blocks<kJ>(v);
 #pragma unroll
-        for (int j = 0; j < kJ; ++j) store4<T, VEC>(dst + (b0 + j) * kBlock + e0, valid[j], v[j]);
+            for (int j = 0; j < kJ; ++j) store4<T, VEC>(dst + j * kBlock, valid[j], v[j]);
+        });
     });
 }
 

@@ -41,41 +41,44 @@ quantize_kernel(const T *x, size_t rows, size_t n, size_t stride, uint8_t *codes
     for_each_unit<kPq>(units, [&](uint32_t g) {
         const uint32_t row = fast_div(g, per_row);
         const size_t b0 = static_cast<size_t>(g - row * per_row.d) * kJq;
-        const T *xr = x + row * stride;
-        uint8_t *cr = codes + row * stride;
-        float v[kJq][4];
-        int valid[kJq];
-        float amax[kJq];
+        with_full((b0 + kJq) * kBlock <= n, [&](auto full) {
+            constexpr bool F = decltype(full)::value;
+            const T *xr = x + row * stride + b0 * kBlock + e0;
+            uint8_t *cr = codes + row * stride + b0 * kBlock + e0;
+            float v[kJq][4];
+            int valid[kJq];
+            float amax[kJq];
 #pragma unroll
-        for (int j = 0; j < kJq; ++j) {
-            valid[j] = lane_valid((b0 + j) * kBlock, n);
-            load4<T, VEC>(xr + (b0 + j) * kBlock + e0, valid[j], v[j]);
-        }
-#pragma unroll
-        for (int j = 0; j < kJq; ++j) amax[j] = warp_amax4(v[j]);
-        Scale sc[kJq];
-        make_scales<kJq>(amax, sc);
-#pragma unroll
-        for (int j = 0; j < kJq; ++j) {
-            const uint32_t q = quant4(v[j], sc[j]);
-            uint8_t *dst = cr + (b0 + j) * kBlock + e0;
-            if (VEC && valid[j] == 4) {
-                st_stream(reinterpret_cast<unsigned int *>(dst), q);
-            } else {
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    if (k < valid[j]) dst[k] = static_cast<uint8_t>(q >> (8 * k));
+            for (int j = 0; j < kJq; ++j) {
+                valid[j] = F ? 4 : lane_valid((b0 + j) * kBlock, n);
+                load4<T, VEC>(xr + j * kBlock, valid[j], v[j]);
             }
-        }
-        // lane j < kJq stores the scale of block b0 + j
-        const int l = lane_id();
-        if (l < kJq && b0 + l < nbr) {
-            float s = sc[0].s;
 #pragma unroll
-            for (int j = 1; j < kJq; ++j)
-                if (l == j) s = sc[j].s;
-            st_stream(scales + row * nbr + b0 + l, s);
-        }
+            for (int j = 0; j < kJq; ++j) amax[j] = warp_amax4(v[j]);
+            Scale sc[kJq];
+            make_scales<kJq>(amax, sc);
+#pragma unroll
+            for (int j = 0; j < kJq; ++j) {
+                const uint32_t q = quant4(v[j], sc[j]);
+                uint8_t *dst = cr + j * kBlock;
+                if (VEC && valid[j] == 4) {
+                    st_stream(reinterpret_cast<unsigned int *>(dst), q);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        if (k < valid[j]) dst[k] = static_cast<uint8_t>(q >> (8 * k));
+                }
+            }
+            // lane j < kJq stores the scale of block b0 + j
+            const int l = lane_id();
+            if (l < kJq && (F || b0 + l < nbr)) {
+                float s = sc[0].s;
+#pragma unroll
+                for (int j = 1; j < kJq; ++j)
+                    if (l == j) s = sc[j].s;
+                st_stream(scales + row * nbr + b0 + l, s);
+            }
+        });
     });
 }
 
@@ -89,33 +92,35 @@ dequantize_kernel(const uint8_t *codes, const float *scales, size_t rows, size_t
     for_each_unit<kPdq>(units, [&](uint32_t g) {
         const uint32_t row = fast_div(g, per_row);
         const size_t b0 = static_cast<size_t>(g - row * per_row.d) * kJd;
-        const uint8_t *cr = codes + row * stride;
-        const float *sr = scales + row * nbr;
-        T *yr = y + row * stride;
-        uint32_t q[kJd];
-        float s[kJd];
-        int valid[kJd];
+        with_full((b0 + kJd) * kBlock <= n, [&](auto full) {
+            constexpr bool F = decltype(full)::value;
+            const uint8_t *cr = codes + row * stride + b0 * kBlock + e0;
+            const float *sr = scales + row * nbr + b0;
+            T *yr = y + row * stride + b0 * kBlock + e0;
+            uint32_t q[kJd];
+            float s[kJd];
+            int valid[kJd];
 #pragma unroll
-        for (int j = 0; j < kJd; ++j) {
-            const size_t b = b0 + j;
-            valid[j] = lane_valid(b * kBlock, n);
-            const uint8_t *src = cr + b * kBlock + e0;
-            q[j] = 0;
-            if (VEC && valid[j] == 4) {
-                q[j] = ld_stream(reinterpret_cast<const unsigned int *>(src));
-            } else {
+            for (int j = 0; j < kJd; ++j) {
+                valid[j] = F ? 4 : lane_valid((b0 + j) * kBlock, n);
+                const uint8_t *src = cr + j * kBlock;
+                q[j] = 0;
+                if (VEC && valid[j] == 4) {
+                    q[j] = ld_stream(reinterpret_cast<const unsigned int *>(src));
+                } else {
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    if (k < valid[j]) q[j] |= static_cast<uint32_t>(src[k]) << (8 * k);
+                    for (int k = 0; k < 4; ++k)
+                        if (k < valid[j]) q[j] |= static_cast<uint32_t>(src[k]) << (8 * k);
+                }
+                s[j] = (F || b0 + j < nbr) ? ld_stream(sr + j) : 0.0f;
             }
-            s[j] = b < nbr ? ld_stream(sr + b) : 0.0f;
-        }
 #pragma unroll
-        for (int j = 0; j < kJd; ++j) {
-            float v[4];
-            dequant4(q[j], s[j], v);
-            store4<T, VEC>(yr + (b0 + j) * kBlock + e0, valid[j], v);
-        }
+            for (int j = 0; j < kJd; ++j) {
+                float v[4];
+                dequant4(q[j], s[j], v);
+                store4<T, VEC>(yr + j * kBlock, valid[j], v);
+            }
+        });
     });
 }
 

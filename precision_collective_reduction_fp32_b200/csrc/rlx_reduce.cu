@@ -30,29 +30,6 @@ namespace {
 
 template <typename T> struct VecN { static constexpr int n = 16 / sizeof(T); };
 
-// V consecutive elements as fp32; `valid` of them real, the rest +0.
-template <typename T, bool VEC>
-__device__ __forceinline__ void loadv(const T *p, int valid, float (&v)[VecN<T>::n]) {
-    constexpr int V = VecN<T>::n;
-    if (VEC && valid == V) {
-        const uint4 q = ld_stream(reinterpret_cast<const uint4 *>(p));
-        if constexpr (sizeof(T) == 4) {
-            v[0] = __uint_as_float(q.x); v[1] = __uint_as_float(q.y);
-            v[2] = __uint_as_float(q.z); v[3] = __uint_as_float(q.w);
-        } else {
-            const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                v[2 * k] = __uint_as_float(w[k] << 16);
-                v[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
-            }
-        }
-    } else {
-#pragma unroll
-        for (int k = 0; k < V; ++k) v[k] = k < valid ? Elem<T>::load(p + k) : 0.0f;
-    }
-}
-
 template <typename T, bool VEC>
 __device__ __forceinline__ void storev(T *p, int valid, const float (&v)[VecN<T>::n]) {
     constexpr int V = VecN<T>::n;
@@ -77,24 +54,57 @@ __device__ __forceinline__ void storev(T *p, int valid, const float (&v)[VecN<T>
     }
 }
 
+// One 16-byte vector kept as raw words (valid elements; the rest +0), so a
+// bf16 vector costs 4 registers, not 8, while all ranks are in flight.
+template <typename T, bool VEC>
+__device__ __forceinline__ uint4 loadv_raw(const T *p, int valid) {
+    constexpr int V = VecN<T>::n;
+    if (VEC && valid == V) return ld_stream(reinterpret_cast<const uint4 *>(p));
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int k = 0; k < V; ++k) {
+        if (k < valid) {
+            if constexpr (sizeof(T) == 4)
+                w[k] = __float_as_uint(Elem<float>::load(reinterpret_cast<const float *>(p) + k));
+            else
+                w[k / 2] |= static_cast<uint32_t>(ld_stream(reinterpret_cast<const unsigned short *>(p) + k))
+                            << (16 * (k % 2));
+        }
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Element k (compile-time) of a raw vector, widened to fp32 exactly.
+template <typename T, int K>
+__device__ __forceinline__ float raw_elem(const uint4 &q) {
+    constexpr int word = sizeof(T) == 4 ? K : K / 2;
+    const uint32_t w = word == 0 ? q.x : word == 1 ? q.y : word == 2 ? q.z : q.w;
+    if constexpr (sizeof(T) == 4) return __uint_as_float(w);
+    else return __uint_as_float(K % 2 == 0 ? w << 16 : w & 0xffff0000u);
+}
+
+template <typename T, int K = 0>
+__device__ __forceinline__ void add_raw(float (&acc)[VecN<T>::n], const uint4 &q, bool first) {
+    if constexpr (K < VecN<T>::n) {
+        const float v = raw_elem<T, K>(q);
+        acc[K] = first ? v : __fadd_rn(acc[K], v);
+        add_raw<T, K + 1>(acc, q, first);
+    }
+}
+
 // acc = x_0 + x_1 + ... + x_{n-1} (rank order) of the vector at `src` in each
 // of the n rows (row pitch `pitch` elements).  All loads are issued first.
 template <typename T, int NR, bool VEC>
 __device__ __forceinline__ void reduce_vec(const T *src, size_t pitch, int n, int valid,
                                            float (&acc)[VecN<T>::n]) {
-    constexpr int V = VecN<T>::n;
-    float x[NR][V];
+    uint4 x[NR];
 #pragma unroll
     for (int s = 0; s < NR; ++s)
-        if (s < n) loadv<T, VEC>(src + s * pitch, valid, x[s]);
-#pragma unroll
-    for (int k = 0; k < V; ++k) acc[k] = x[0][k];
+        if (s < n) x[s] = loadv_raw<T, VEC>(src + s * pitch, valid);
+    add_raw<T>(acc, x[0], true);
 #pragma unroll
     for (int s = 1; s < NR; ++s)
-        if (s < n) {
-#pragma unroll
-            for (int k = 0; k < V; ++k) acc[k] = __fadd_rn(acc[k], x[s][k]);
-        }
+        if (s < n) add_raw<T>(acc, x[s], false);
 }
 
 // ---------------------------------------------------- FP8 wire, warp per block
@@ -138,6 +148,18 @@ __device__ __forceinline__ void reduce_block_fp8(const T *src, size_t pitch, int
 constexpr int kPn = RLX_P_NATIVE;
 constexpr int kPf = RLX_P_FP8;
 
+// Valid elements of a vector starting at element i0 of a segment ending at
+// `hi` (V when the unit is full).
+template <int V, typename Full>
+__device__ __forceinline__ int vec_valid_in(size_t i0, size_t hi, Full) {
+    if constexpr (Full::value) {
+        return V;
+    } else {
+        if (i0 >= hi) return 0;
+        return hi - i0 < static_cast<size_t>(V) ? static_cast<int>(hi - i0) : V;
+    }
+}
+
 // DDA-flat, native: unit g = 32 consecutive 16-byte vectors (lane l: 32g + l).
 template <typename T, int NR, bool VEC>
 __global__ void __launch_bounds__(kThreads)
@@ -146,13 +168,14 @@ flat_native_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
     const size_t nvec = (count + V - 1) / V;
     const uint32_t units = static_cast<uint32_t>((nvec + 31) / 32);
     for_each_unit<kPn>(units, [&](uint32_t g) {
-        const size_t v = static_cast<size_t>(g) * 32 + lane_id();
-        if (v >= nvec) return;
-        const size_t i0 = v * V;
-        const int valid = count - i0 < static_cast<size_t>(V) ? static_cast<int>(count - i0) : V;
-        float acc[V];
-        reduce_vec<T, NR, VEC>(send + i0, stride, n, valid, acc);
-        for (int r = 0; r < n; ++r) storev<T, VEC>(recv + r * stride + i0, valid, acc);
+        const size_t i0 = (static_cast<size_t>(g) * 32 + lane_id()) * V;
+        with_full((static_cast<size_t>(g) + 1) * 32 * V <= count, [&](auto full) {
+            const int valid = vec_valid_in<V>(i0, count, full);
+            if (valid == 0) return;
+            float acc[V];
+            reduce_vec<T, NR, VEC>(send + i0, stride, n, valid, acc);
+            for (int r = 0; r < n; ++r) storev<T, VEC>(recv + r * stride + i0, valid, acc);
+        });
     });
 }
 
@@ -164,10 +187,12 @@ flat_fp8_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
     const int e0 = lane_id() * 4;
     for_each_unit<kPf>(nblk, [&](uint32_t b) {
         const size_t base = static_cast<size_t>(b) * kBlock;
-        const int valid = lane_valid(base, count);
-        float acc[4];
-        reduce_block_fp8<T, NR, VEC>(send + base, stride, n, valid, acc);
-        for (int r = 0; r < n; ++r) store4<T, VEC>(recv + r * stride + base + e0, valid, acc);
+        with_full(base + kBlock <= count, [&](auto full) {
+            const int valid = decltype(full)::value ? 4 : lane_valid(base, count);
+            float acc[4];
+            reduce_block_fp8<T, NR, VEC>(send + base, stride, n, valid, acc);
+            for (int r = 0; r < n; ++r) store4<T, VEC>(recv + r * stride + base + e0, valid, acc);
+        });
     });
 }
 
@@ -182,13 +207,16 @@ tree_reduce_native_kernel(const T *send, T *recv, size_t count, size_t stride, i
         const uint32_t c = fast_div(g, per_chunk);
         const size_t lo = static_cast<size_t>(c) * chunk;
         if (lo >= count) return;
-        const size_t i0 = lo + (static_cast<size_t>(g - c * per_chunk.d) * 32 + lane_id()) * V;
         const size_t hi = count - lo < chunk ? count : lo + chunk;
-        if (i0 >= hi) return;
-        const int valid = hi - i0 < static_cast<size_t>(V) ? static_cast<int>(hi - i0) : V;
-        float acc[V];
-        reduce_vec<T, NR, VEC>(send + i0, stride, n, valid, acc);
-        storev<T, VEC>(recv + c * stride + i0, valid, acc);
+        const size_t u0 = lo + static_cast<size_t>(g - c * per_chunk.d) * 32 * V;
+        const size_t i0 = u0 + static_cast<size_t>(lane_id()) * V;
+        with_full(u0 + 32 * V <= hi, [&](auto full) {
+            const int valid = vec_valid_in<V>(i0, hi, full);
+            if (valid == 0) return;
+            float acc[V];
+            reduce_vec<T, NR, VEC>(send + i0, stride, n, valid, acc);
+            storev<T, VEC>(recv + c * stride + i0, valid, acc);
+        });
     });
 }
 
@@ -203,13 +231,16 @@ tree_reduce_fp8_kernel(const T *send, size_t count, size_t stride, int n,
     const int e0 = lane_id() * 4;
     for_each_unit<kPf>(nblk, [&](uint32_t b) {
         const size_t base = static_cast<size_t>(b) * kBlock;
-        float acc[4];
-        reduce_block_fp8<T, NR, VEC>(send + base, stride, n, lane_valid(base, count), acc);
-        const Scale sc = make_scale(warp_amax4(acc));
-        const uint32_t codes = quant4(acc, sc);
-        // default caching: pass 2 reads the payload back right away
-        *reinterpret_cast<uint32_t *>(ws_codes + base + e0) = codes;
-        if (lane_id() == 0) ws_scales[b] = sc.s;
+        with_full(base + kBlock <= count, [&](auto full) {
+            const int valid = decltype(full)::value ? 4 : lane_valid(base, count);
+            float acc[4];
+            reduce_block_fp8<T, NR, VEC>(send + base, stride, n, valid, acc);
+            const Scale sc = make_scale(warp_amax4(acc));
+            const uint32_t codes = quant4(acc, sc);
+            // default caching: pass 2 reads the payload back right away
+            *reinterpret_cast<uint32_t *>(ws_codes + base + e0) = codes;
+            if (lane_id() == 0) ws_scales[b] = sc.s;
+        });
     });
 }
 
@@ -222,12 +253,15 @@ rs_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t 
     const uint32_t units = per_chunk.d * static_cast<uint32_t>(n);
     for_each_unit<kPn>(units, [&](uint32_t g) {
         const uint32_t r = fast_div(g, per_chunk);
-        const size_t j0 = (static_cast<size_t>(g - r * per_chunk.d) * 32 + lane_id()) * V;
-        if (j0 >= m) return;
-        const int valid = m - j0 < static_cast<size_t>(V) ? static_cast<int>(m - j0) : V;
-        float acc[V];
-        reduce_vec<T, NR, VEC>(send + r * m + j0, sstride, n, valid, acc);
-        storev<T, VEC>(recv + r * rstride + j0, valid, acc);
+        const size_t u0 = static_cast<size_t>(g - r * per_chunk.d) * 32 * V;
+        const size_t j0 = u0 + static_cast<size_t>(lane_id()) * V;
+        with_full(u0 + 32 * V <= m, [&](auto full) {
+            const int valid = vec_valid_in<V>(j0, m, full);
+            if (valid == 0) return;
+            float acc[V];
+            reduce_vec<T, NR, VEC>(send + r * m + j0, sstride, n, valid, acc);
+            storev<T, VEC>(recv + r * rstride + j0, valid, acc);
+        });
     });
 }
 
@@ -242,10 +276,12 @@ rs_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, 
     for_each_unit<kPf>(units, [&](uint32_t g) {
         const uint32_t r = fast_div(g, per_chunk);
         const size_t j0 = static_cast<size_t>(g - r * per_chunk.d) * kBlock;
-        const int valid = lane_valid(j0, m);
-        float acc[4];
-        reduce_block_fp8<T, NR, VEC>(send + r * m + j0, sstride, n, valid, acc);
-        store4<T, VEC>(recv + r * rstride + j0 + e0, valid, acc);
+        with_full(j0 + kBlock <= m, [&](auto full) {
+            const int valid = decltype(full)::value ? 4 : lane_valid(j0, m);
+            float acc[4];
+            reduce_block_fp8<T, NR, VEC>(send + r * m + j0, sstride, n, valid, acc);
+            store4<T, VEC>(recv + r * rstride + j0 + e0, valid, acc);
+        });
     });
 }
 
