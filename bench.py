@@ -78,6 +78,33 @@ OPS = list(op_bytes(COUNT, NRANKS).keys())
 KERNELS_PER_OP = {op: (2 if op.startswith("allreduce_tree") else 1) for op in OPS}
 
 
+# ------------------------------------------------------------ multi-GPU host
+
+def gpu_seed(sim_rank: int, gpu_rank: int) -> int:
+    """Seed of simulated rank `sim_rank` in the batch of GPU `gpu_rank`: every
+    GPU works on its own independent batch (weak scaling, no exchange)."""
+    from precision_collective_reduction_fp32_b200 import synth
+    return synth.seed(WORKLOAD, sim_rank) + 100 * gpu_rank
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """The maximum of x over all processes of the default group (x itself
+    when there is no group).  Timings are reported as the slowest rank."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(world: int, bytes_per_step: int, steps: int, ms: float) -> float:
+    """Effective GB/s of all GPUs together: every GPU moved bytes_per_step per
+    step, the job took `ms` (the slowest GPU)."""
+    return world * bytes_per_step * steps / (ms * 1e-3) / 1e9
+
+
 # ------------------------------------------------------------------ helpers
 
 def peaks() -> tuple[float, str]:
@@ -233,7 +260,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
     count = args.count
     x_host = np.empty((NRANKS, count), dtype=np.float32)
     for r in range(NRANKS):
-        x_host[r] = synth.draw_row("normal_outliers", count, synth.seed(WORKLOAD, r) + 100 * rank)
+        x_host[r] = synth.draw_row("normal_outliers", count, gpu_seed(r, rank))
     step = Step(x_host, dev)
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream or None
@@ -274,11 +301,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
     for k in range(K):
         for i, (name, _) in enumerate(ops):
             per_op_ms[name] += ev[k][i].elapsed_time(ev[k][i + 1])
-    total_ms = ev[0][0].elapsed_time(ev[K - 1][-1])
-    t_dev = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_dev, op=dist.ReduceOp.MAX)
-    total_ms = float(t_dev.item())
+    total_ms = max_over_ranks(ev[0][0].elapsed_time(ev[K - 1][-1]), dev)
 
     # ---- end to end: pinned host -> device, the step, result -> host
     host_in = torch.from_numpy(x_host).pin_memory()
@@ -301,16 +324,13 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         host_out.copy_(out_dev, non_blocking=True)   # the FP8 tree allreduce result
     e1.record(stream)
     torch.cuda.synchronize()
-    e_dev = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e_dev, op=dist.ReduceOp.MAX)
-    e2e_ms = float(e_dev.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     barrier()
     if rank != 0:
         return None
 
     peak, peak_kind = peaks()
-    value = world * step_bytes * K / (total_ms * 1e-3) / 1e9
+    value = whole_job_gbs(world, step_bytes, K, total_ms)
     per_op = {}
     for name in per_op_ms:
         ms = per_op_ms[name] / K
@@ -351,7 +371,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
                      "algorithmic_bytes": bytes_[dom], "peak_kind": peak_kind},
         "gpu_launches": K * sum(KERNELS_PER_OP[n] for n in bytes_),
         "clocks": clk,
-        "e2e": {"value": round(world * step_bytes * Ke / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+        "e2e": {"value": round(whole_job_gbs(world, step_bytes, Ke, e2e_ms), 1), "unit": "GB/s",
                 "h2d_bytes_per_step": NRANKS * count * 4, "d2h_bytes_per_step": NRANKS * count * 4,
                 "ms_per_step": round(e2e_ms / Ke, 3), "steps": Ke},
     }

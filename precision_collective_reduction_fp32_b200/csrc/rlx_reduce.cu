@@ -93,18 +93,29 @@ __device__ __forceinline__ void add_raw(float (&acc)[VecN<T>::n], const uint4 &q
 }
 
 // acc = x_0 + x_1 + ... + x_{n-1} (rank order) of the vector at `src` in each
-// of the n rows (row pitch `pitch` elements).  All loads are issued first.
-template <typename T, int NR, bool VEC>
-__device__ __forceinline__ void reduce_vec(const T *src, size_t pitch, int n, int valid,
+// of the n rows (row pitch `pitch` elements).  Full vectors issue all n loads
+// before the first add; a partial (tail) vector is summed rank by rank, which
+// needs few registers and keeps the kernel's register budget for the hot path.
+template <typename T, int NR, bool VEC, typename Full>
+__device__ __forceinline__ void reduce_vec(const T *src, size_t pitch, int n, int valid, Full,
                                            float (&acc)[VecN<T>::n]) {
-    uint4 x[NR];
+    if constexpr (Full::value) {
+        uint4 x[NR];
+        const T *p = src;   // one running pointer: no per-rank address registers
 #pragma unroll
-    for (int s = 0; s < NR; ++s)
-        if (s < n) x[s] = loadv_raw<T, VEC>(src + s * pitch, valid);
-    add_raw<T>(acc, x[0], true);
+        for (int s = 0; s < NR; ++s) {
+            if (s < n) x[s] = loadv_raw<T, VEC>(p, valid);
+            p += pitch;
+        }
+        add_raw<T>(acc, x[0], true);
 #pragma unroll
-    for (int s = 1; s < NR; ++s)
-        if (s < n) add_raw<T>(acc, x[s], false);
+        for (int s = 1; s < NR; ++s)
+            if (s < n) add_raw<T>(acc, x[s], false);
+    } else {
+        add_raw<T>(acc, loadv_raw<T, false>(src, valid), true);
+#pragma unroll 1
+        for (int s = 1; s < n; ++s) add_raw<T>(acc, loadv_raw<T, false>(src + s * pitch, valid), false);
+    }
 }
 
 // ---------------------------------------------------- FP8 wire, warp per block
@@ -148,6 +159,18 @@ __device__ __forceinline__ void reduce_block_fp8(const T *src, size_t pitch, int
 constexpr int kPn = RLX_P_NATIVE;
 constexpr int kPf = RLX_P_FP8;
 
+// Resident CTAs per SM requested from the compiler (caps registers per
+// thread) for kernels with up to 8 ranks; the 16-rank forms hold twice the
+// data and get the default.
+#ifndef RLX_MINB_NATIVE
+#define RLX_MINB_NATIVE 5
+#endif
+#ifndef RLX_MINB_FP8
+#define RLX_MINB_FP8 3
+#endif
+template <int NR> constexpr int kMinBlocksNative = NR <= 8 ? RLX_MINB_NATIVE : 1;
+template <int NR> constexpr int kMinBlocksFp8 = NR <= 8 ? RLX_MINB_FP8 : 1;
+
 // Valid elements of a vector starting at element i0 of a segment ending at
 // `hi` (V when the unit is full).
 template <int V, typename Full>
@@ -162,7 +185,7 @@ __device__ __forceinline__ int vec_valid_in(size_t i0, size_t hi, Full) {
 
 // DDA-flat, native: unit g = 32 consecutive 16-byte vectors (lane l: 32g + l).
 template <typename T, int NR, bool VEC>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, kMinBlocksNative<NR>)
 flat_native_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
     constexpr int V = VecN<T>::n;
     const size_t nvec = (count + V - 1) / V;
@@ -173,7 +196,7 @@ flat_native_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
             const int valid = vec_valid_in<V>(i0, count, full);
             if (valid == 0) return;
             float acc[V];
-            reduce_vec<T, NR, VEC>(send + i0, stride, n, valid, acc);
+            reduce_vec<T, NR, VEC>(send + i0, stride, n, valid, full, acc);
             for (int r = 0; r < n; ++r) storev<T, VEC>(recv + r * stride + i0, valid, acc);
         });
     });
@@ -181,7 +204,7 @@ flat_native_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
 
 // DDA-flat, FP8: unit g = 128-block g.
 template <typename T, int NR, bool VEC>
-__global__ void __launch_bounds__(kThreads, NR <= 8 ? 3 : 1)
+__global__ void __launch_bounds__(kThreads, kMinBlocksFp8<NR>)
 flat_fp8_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
     const uint32_t nblk = static_cast<uint32_t>((count + kBlock - 1) / kBlock);
     const int e0 = lane_id() * 4;
@@ -198,7 +221,7 @@ flat_fp8_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
 
 // DDA-tree pass 1, native: unit = (chunk c, 32 vectors of it); chunk c -> row c.
 template <typename T, int NR, bool VEC>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, kMinBlocksNative<NR>)
 tree_reduce_native_kernel(const T *send, T *recv, size_t count, size_t stride, int n,
                           size_t chunk, FastDiv per_chunk) {
     constexpr int V = VecN<T>::n;
@@ -214,7 +237,7 @@ tree_reduce_native_kernel(const T *send, T *recv, size_t count, size_t stride, i
             const int valid = vec_valid_in<V>(i0, hi, full);
             if (valid == 0) return;
             float acc[V];
-            reduce_vec<T, NR, VEC>(send + i0, stride, n, valid, acc);
+            reduce_vec<T, NR, VEC>(send + i0, stride, n, valid, full, acc);
             storev<T, VEC>(recv + c * stride + i0, valid, acc);
         });
     });
@@ -224,7 +247,7 @@ tree_reduce_native_kernel(const T *send, T *recv, size_t count, size_t stride, i
 // block again into the workspace payload (codes padded to whole blocks, one
 // scale per block).
 template <typename T, int NR, bool VEC>
-__global__ void __launch_bounds__(kThreads, NR <= 8 ? 3 : 1)
+__global__ void __launch_bounds__(kThreads, kMinBlocksFp8<NR>)
 tree_reduce_fp8_kernel(const T *send, size_t count, size_t stride, int n,
                        uint8_t *ws_codes, float *ws_scales) {
     const uint32_t nblk = static_cast<uint32_t>((count + kBlock - 1) / kBlock);
@@ -246,7 +269,7 @@ tree_reduce_fp8_kernel(const T *send, size_t count, size_t stride, int n,
 
 // ReduceScatter, native: unit = (destination rank r, 32 vectors of chunk r).
 template <typename T, int NR, bool VEC>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, kMinBlocksNative<NR>)
 rs_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n,
                  FastDiv per_chunk) {
     constexpr int V = VecN<T>::n;
@@ -259,7 +282,7 @@ rs_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t 
             const int valid = vec_valid_in<V>(j0, m, full);
             if (valid == 0) return;
             float acc[V];
-            reduce_vec<T, NR, VEC>(send + r * m + j0, sstride, n, valid, acc);
+            reduce_vec<T, NR, VEC>(send + r * m + j0, sstride, n, valid, full, acc);
             storev<T, VEC>(recv + r * rstride + j0, valid, acc);
         });
     });
@@ -268,7 +291,7 @@ rs_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t 
 // ReduceScatter, FP8: unit = (destination rank r, 128-block of chunk r);
 // blocks anchored at the chunk start r*m.
 template <typename T, int NR, bool VEC>
-__global__ void __launch_bounds__(kThreads, NR <= 8 ? 3 : 1)
+__global__ void __launch_bounds__(kThreads, kMinBlocksFp8<NR>)
 rs_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n,
               FastDiv per_chunk) {
     const uint32_t units = per_chunk.d * static_cast<uint32_t>(n);
