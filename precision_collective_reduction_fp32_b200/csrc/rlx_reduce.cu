@@ -163,13 +163,17 @@ constexpr int kPf = RLX_P_FP8;
 // thread) for kernels with up to 8 ranks; the 16-rank forms hold twice the
 // data and get the default.
 #ifndef RLX_MINB_NATIVE
-#define RLX_MINB_NATIVE 5
+#define RLX_MINB_NATIVE 3
 #endif
 #ifndef RLX_MINB_FP8
-#define RLX_MINB_FP8 3
+#define RLX_MINB_FP8 4
+#endif
+#ifndef RLX_MINB_FP8_FLAT
+#define RLX_MINB_FP8_FLAT 3
 #endif
 template <int NR> constexpr int kMinBlocksNative = NR <= 8 ? RLX_MINB_NATIVE : 1;
 template <int NR> constexpr int kMinBlocksFp8 = NR <= 8 ? RLX_MINB_FP8 : 1;
+template <int NR> constexpr int kMinBlocksFp8Flat = NR <= 8 ? RLX_MINB_FP8_FLAT : 1;
 
 // Valid elements of a vector starting at element i0 of a segment ending at
 // `hi` (V when the unit is full).
@@ -204,7 +208,7 @@ flat_native_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
 
 // DDA-flat, FP8: unit g = 128-block g.
 template <typename T, int NR, bool VEC>
-__global__ void __launch_bounds__(kThreads, kMinBlocksFp8<NR>)
+__global__ void __launch_bounds__(kThreads, kMinBlocksFp8Flat<NR>)
 flat_fp8_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
     const uint32_t nblk = static_cast<uint32_t>((count + kBlock - 1) / kBlock);
     const int e0 = lane_id() * 4;
