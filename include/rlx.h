@@ -170,6 +170,33 @@ RLX_API rlx_status rlx_alltoall(const void *send, size_t send_stride, void *recv
                         size_t recv_stride, size_t m, int nranks, rlx_dtype dtype,
                         rlx_wire wire, void *stream);
 
+/*
+ * DDA-tree SUM allreduce without a workspace argument, for callers that
+ * cannot allocate device memory where they run the collective (a plug-in
+ * handed only its input and output buffers, or a loop that must not call
+ * cudaMalloc because it can synchronise the whole device).  The pages have
+ * no counterpart: this is a convenience of this library.
+ *
+ * Same arguments and results as rlx_allreduce_tree, bit for bit.  On the FP8
+ * wire the payload between the two passes lives in a fixed device array that
+ * the library defines at file scope (16.5 MiB on every GPU that loads the
+ * library, held until the process exits), so count may be at most
+ * RLX_NOALLOC_MAX_COUNT elements per rank; larger counts return
+ * RLX_ERR_WORKSPACE and launch nothing.  The native wire needs no payload
+ * and has no such limit.  The library allocates nothing.
+ *
+ * The first call on each device looks up the array's device address with
+ * that device current; make that first call before any stream capture.
+ * All calls on a device share the one array: two calls whose kernels can
+ * overlap on the GPU (different streams, no ordering between them) race on
+ * it.  Calls ordered on one stream are safe; nothing in the array needs to
+ * be cleared between calls.
+ */
+#define RLX_NOALLOC_MAX_COUNT 16777216u
+RLX_API rlx_status rlx_allreduce_tree_noalloc(const void *send, void *recv, size_t count,
+                                              size_t stride, int nranks, rlx_dtype dtype,
+                                              rlx_wire wire, rlx_op op, void *stream);
+
 /* Workspace bytes the collective needs for these arguments (0 = none). */
 RLX_API size_t rlx_workspace_bytes(rlx_coll coll, size_t count, int nranks, rlx_dtype dtype,
                            rlx_wire wire);

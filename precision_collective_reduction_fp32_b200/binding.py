@@ -26,7 +26,8 @@ RLX_MAX_RANKS = 16
 # every symbol include/rlx.h declares
 EXPORTS = ("rlx_quantize_fp8", "rlx_dequantize_fp8", "rlx_allreduce_flat", "rlx_allreduce_tree",
            "rlx_reduce_scatter", "rlx_all_gather", "rlx_alltoall", "rlx_workspace_bytes",
-           "rlx_status_string", "rlx_last_cuda_error")
+           "rlx_status_string", "rlx_last_cuda_error", "rlx_allreduce_tree_noalloc")
+RLX_NOALLOC_MAX_COUNT = 16777216
 
 
 class RlxError(RuntimeError):
@@ -55,6 +56,7 @@ def lib() -> ctypes.CDLL:
             "rlx_dequantize_fp8": [P, P, S, S, S, P, I, P],
             "rlx_allreduce_flat": [P, P, S, S, I, I, I, I, P],
             "rlx_allreduce_tree": [P, P, S, S, I, I, I, I, P, S, P],
+            "rlx_allreduce_tree_noalloc": [P, P, S, S, I, I, I, I, P],
             "rlx_reduce_scatter": [P, S, P, S, S, I, I, I, I, P],
             "rlx_all_gather": [P, S, P, S, S, I, I, I, P],
             "rlx_alltoall": [P, S, P, S, S, I, I, I, P],
@@ -111,6 +113,14 @@ def rlx_allreduce_tree(send, recv, count, stride, nranks, dtype, wire, op=RLX_SU
                        workspace=None, workspace_bytes=0, stream=None) -> None:
     _call("rlx_allreduce_tree", send, recv, count, stride, nranks, dtype, wire, op, workspace,
           workspace_bytes, stream)
+
+
+def rlx_allreduce_tree_noalloc(send, recv, count, stride, nranks, dtype, wire, op=RLX_SUM,
+                               stream=None) -> None:
+    """DDA-tree allreduce whose FP8 payload sits in the library's fixed
+    device array (no workspace argument; count <= RLX_NOALLOC_MAX_COUNT on
+    the FP8 wire).  For callers that cannot allocate device memory."""
+    _call("rlx_allreduce_tree_noalloc", send, recv, count, stride, nranks, dtype, wire, op, stream)
 
 
 def rlx_reduce_scatter(send, send_stride, recv, recv_stride, m, nranks, dtype, wire,

@@ -55,6 +55,12 @@ rlx_status from_cuda(cudaError_t e) {
     return RLX_ERR_CUDA;
 }
 
+}  // namespace
+
+void rlx::record_cuda_error(cudaError_t e) { g_last_cuda_error = static_cast<int>(e); }
+
+namespace {
+
 size_t elem_size(rlx_dtype d) { return d == RLX_BF16 ? 2 : 4; }
 
 bool dtype_ok(rlx_dtype d) { return d == RLX_F32 || d == RLX_BF16; }

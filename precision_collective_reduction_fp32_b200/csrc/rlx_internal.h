@@ -20,6 +20,9 @@ constexpr int kThreads = 256;  // threads per CTA for every kernel
 // an empty grid.
 dim3 grid_for(const void *kernel, size_t units, size_t units_per_cta);
 
+// Records a CUDA failure for rlx_last_cuda_error() of the calling thread.
+void record_cuda_error(cudaError_t e);
+
 // DDA-flat, all wires.  nranks >= 2.
 cudaError_t launch_allreduce_flat(const void *send, void *recv, size_t count, size_t stride,
                                   int nranks, rlx_dtype dtype, rlx_wire wire, bool vec,
