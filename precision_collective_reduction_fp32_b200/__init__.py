@@ -13,6 +13,8 @@ path: without librlx.so every call raises.
 """
 from __future__ import annotations
 
+import os
+
 import torch
 
 from . import binding as _b
@@ -20,13 +22,15 @@ from .binding import (RLX_BF16, RLX_BLOCK, RLX_COLL_ALL_GATHER, RLX_COLL_ALLREDU
                       RLX_COLL_ALLREDUCE_TREE, RLX_COLL_ALLTOALL, RLX_COLL_REDUCE_SCATTER,
                       RLX_F32, RLX_MAX_RANKS, RLX_SUM, RLX_WIRE_FP8_E4M3, RLX_WIRE_NATIVE,
                       RlxError, rlx_all_gather, rlx_allreduce_flat, rlx_allreduce_tree,
-                      rlx_alltoall, rlx_dequantize_fp8, rlx_quantize_fp8, rlx_reduce_scatter,
-                      rlx_status_string, rlx_workspace_bytes)
+                      rlx_allreduce_tree_noalloc, rlx_alltoall, rlx_dequantize_fp8,
+                      rlx_quantize_fp8, rlx_reduce_scatter, rlx_status_string,
+                      rlx_workspace_bytes)
 
 __all__ = ["allreduce", "reduce_scatter", "all_gather", "alltoall", "quantize_fp8",
            "dequantize_fp8", "workspace_bytes", "RlxError", "rlx_allreduce_flat",
-           "rlx_allreduce_tree", "rlx_reduce_scatter", "rlx_all_gather", "rlx_alltoall",
-           "rlx_quantize_fp8", "rlx_dequantize_fp8", "rlx_workspace_bytes", "rlx_status_string"]
+           "rlx_allreduce_tree", "rlx_allreduce_tree_noalloc", "rlx_reduce_scatter",
+           "rlx_all_gather", "rlx_alltoall", "rlx_quantize_fp8", "rlx_dequantize_fp8",
+           "rlx_workspace_bytes", "rlx_status_string", "default_wire"]
 
 _WIRES = {"native": RLX_WIRE_NATIVE, "fp8": RLX_WIRE_FP8_E4M3}
 
@@ -64,19 +68,35 @@ def ctypes_stream(s: torch.cuda.Stream):
     return s.cuda_stream or None
 
 
-def _wire(w: str) -> int:
+# The pages switch the low-precision collectives on for a whole job with an
+# environment variable ("Coletivos de Baixa Precisão", infolabhq pt:
+# RCCL_LOW_PRECISION_ENABLE=1) and let users enable them selectively.  Here a
+# call with wire=None takes the FP8 wire when RLX_LOW_PRECISION_ENABLE (or
+# the pages' RCCL_LOW_PRECISION_ENABLE) is "1", else the native wire; an
+# explicit wire= always wins.
+LOW_PRECISION_ENV = ("RLX_LOW_PRECISION_ENABLE", "RCCL_LOW_PRECISION_ENABLE")
+
+
+def default_wire() -> str:
+    return "fp8" if any(os.environ.get(v) == "1" for v in LOW_PRECISION_ENV) else "native"
+
+
+def _wire(w: str | None) -> int:
+    if w is None:
+        w = default_wire()
     try:
         return _WIRES[w]
     except KeyError:
         raise ValueError("wire must be 'native' or 'fp8'") from None
 
 
-def workspace_bytes(coll: int, count: int, nranks: int, dtype: torch.dtype, wire: str) -> int:
+def workspace_bytes(coll: int, count: int, nranks: int, dtype: torch.dtype,
+                    wire: str | None = None) -> int:
     d = RLX_F32 if dtype == torch.float32 else RLX_BF16
     return rlx_workspace_bytes(coll, count, nranks, d, _wire(wire))
 
 
-def allreduce(x: torch.Tensor, algo: str = "flat", wire: str = "native",
+def allreduce(x: torch.Tensor, algo: str = "flat", wire: str | None = None,
               out: torch.Tensor | None = None, workspace: torch.Tensor | None = None):
     """SUM allreduce over the ranks (rows) of x.  out may be x (in place)."""
     n, count, stride = _rows(x)
@@ -99,7 +119,7 @@ def allreduce(x: torch.Tensor, algo: str = "flat", wire: str = "native",
     return out
 
 
-def reduce_scatter(x: torch.Tensor, wire: str = "native", out: torch.Tensor | None = None):
+def reduce_scatter(x: torch.Tensor, wire: str | None = None, out: torch.Tensor | None = None):
     """x [N, N*m] -> [N, m]: rank r gets the SUM over ranks of chunk r."""
     n, per, stride = _rows(x)
     if n == 0 or per % n:
@@ -111,7 +131,7 @@ def reduce_scatter(x: torch.Tensor, wire: str = "native", out: torch.Tensor | No
     return out
 
 
-def all_gather(x: torch.Tensor, wire: str = "native", out: torch.Tensor | None = None):
+def all_gather(x: torch.Tensor, wire: str | None = None, out: torch.Tensor | None = None):
     """x [N, m] -> [N, N*m]: every rank gets every rank's chunk."""
     n, m, stride = _rows(x)
     out = torch.empty((n, n * m), dtype=x.dtype, device=x.device) if out is None else out
@@ -120,7 +140,7 @@ def all_gather(x: torch.Tensor, wire: str = "native", out: torch.Tensor | None =
     return out
 
 
-def alltoall(x: torch.Tensor, wire: str = "native", out: torch.Tensor | None = None):
+def alltoall(x: torch.Tensor, wire: str | None = None, out: torch.Tensor | None = None):
     """x [N, N*m] -> [N, N*m]: chunk r of rank s lands at chunk s of rank r."""
     n, per, stride = _rows(x)
     if n == 0 or per % n:

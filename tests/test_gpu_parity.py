@@ -121,6 +121,38 @@ def test_e4m3_hardware_conversion_band():
             assert _bits_equal(got, ref), hex(first)
 
 
+def test_e4m3_hardware_conversion_below_band():
+    """Every fp32 magnitude below 2^-12 (subnormals included), both signs,
+    through the quantiser with block scale 1: the oracle maps all of them to
+    a signed zero (pinned against torch and brute force); the GPU must give
+    0x00 / 0x80 for every one, the oracle's code, checked here on runs spread
+    over the range."""
+    hi = 0x39800000
+    step = 127 * (1 << 17)
+    for sign_bit in (0, 0x80000000):
+        for start in range(0, hi, step):
+            n = min(step, hi - start)
+            nblk = (n + 126) // 127
+            bits = torch.arange(start, start + nblk * 127, dtype=torch.int64, device="cuda")
+            bits = torch.where(bits < start + n, bits, torch.zeros_like(bits)) | sign_bit
+            vals = (bits - (1 << 32) if sign_bit else bits).to(torch.int32).view(torch.float32)
+            blk = torch.empty((nblk, 128), dtype=torch.float32, device="cuda")
+            blk[:, 0] = 448.0
+            blk[:, 1:] = vals.view(nblk, 127)
+            codes = torch.empty((1, nblk * 128), dtype=torch.uint8, device="cuda")
+            scales = torch.empty((1, nblk), dtype=torch.float32, device="cuda")
+            B.rlx_quantize_fp8(blk.data_ptr(), B.RLX_F32, 1, nblk * 128, nblk * 128,
+                               codes.data_ptr(), scales.data_ptr(), stream())
+            torch.cuda.synchronize()
+            assert bool((scales == 1.0).all())
+            body = codes.view(nblk, 128)[:, 1:]
+            assert bool((body == (0x80 if sign_bit else 0)).all()), hex(start | sign_bit)
+        # the value the GPU is held to is the oracle's: runs of the same range
+        for first in range(0, hi, hi // 16):
+            ref = oracle.e4m3_encode_bits_range(sign_bit | first, 1 << 16)
+            assert bool((ref == (0x80 if sign_bit else 0)).all())
+
+
 # ------------------------------------------------------------------ allreduce
 
 AR_CASES = [(n, c) for n in (2, 3, 8) for c in (1, 7, 127, 128, 129, 1000, 3 * 128 * 8 + 5)] + \
