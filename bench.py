@@ -396,11 +396,80 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
                 "ms_per_step": round(e2e_ms / Ke, 3), "steps": Ke,
                 "overlap": "uploads, kernels and downloads on three streams, two device batches"},
     }
+    if world == 1 and not args.only and not args.no_latency:
+        res["small_messages"] = small_message_latency(dev)
     if count != COUNT or args.only:
         res["config"]["workload"] = "PROFILING CASE, not the benchmark: %s on N=8 x fp32[%d]" % (
             ",".join(bytes_), count)
     if world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(x_host, sample=min(CPU_SAMPLE, count))
+    return res
+
+
+# ------------------------------------------------------------ small messages
+
+def small_message_latency(dev, reps: int = 200, graph_reps: int = 50) -> dict:
+    """Microseconds per call for the small-message workloads (decode-sized
+    bf16 [32, 8192] x 8 ranks, and the [10, 20] fp32 quick-start shape), L2
+    hot: back-to-back calls timed with CUDA events, once launched one by one
+    from Python through the C ABI and once replayed from a CUDA graph (no
+    host launch cost)."""
+    import torch
+    from precision_collective_reduction_fp32_b200 import binding as B
+    from precision_collective_reduction_fp32_b200 import synth
+    res = {}
+    cases = [("decode_bf16_8x32x8192", 2, torch.bfloat16, B.RLX_BF16),
+             ("tiny_fp32_8x10x20", 1, torch.float32, B.RLX_F32)]
+    for name, wl, tdt, dcode in cases:
+        xh = synth.rank_buffers(wl)
+        x = torch.from_numpy(xh.view(np.int16) if tdt == torch.bfloat16 else xh).to(dev)
+        x = x.view(tdt) if tdt == torch.bfloat16 else x
+        n, c = x.shape
+        out = torch.empty_like(x)
+        ws = torch.empty(max(B.rlx_workspace_bytes(B.RLX_COLL_ALLREDUCE_TREE, c, n, dcode,
+                                                   B.RLX_WIRE_FP8_E4M3), 16),
+                         dtype=torch.uint8, device=dev)
+        row = {}
+        for algo in ("flat", "tree"):
+            for wname, wire in (("native", B.RLX_WIRE_NATIVE), ("fp8", B.RLX_WIRE_FP8_E4M3)):
+                def call(stream_ptr):
+                    if algo == "flat":
+                        B.rlx_allreduce_flat(x.data_ptr(), out.data_ptr(), c, c, n, dcode, wire,
+                                             B.RLX_SUM, stream_ptr)
+                    else:
+                        B.rlx_allreduce_tree(x.data_ptr(), out.data_ptr(), c, c, n, dcode, wire,
+                                             B.RLX_SUM, ws.data_ptr(), ws.numel(), stream_ptr)
+                st = torch.cuda.current_stream(dev)
+                for _ in range(20):
+                    call(st.cuda_stream or None)
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(st)
+                for _ in range(reps):
+                    call(st.cuda_stream or None)
+                e1.record(st)
+                torch.cuda.synchronize()
+                direct = e0.elapsed_time(e1) / reps * 1e3
+                g = torch.cuda.CUDAGraph()
+                cs = torch.cuda.Stream(dev)
+                with torch.cuda.stream(cs):
+                    call(cs.cuda_stream)
+                    torch.cuda.synchronize()
+                    with torch.cuda.graph(g, stream=cs):
+                        for _ in range(graph_reps):
+                            call(cs.cuda_stream)
+                g.replay()
+                torch.cuda.synchronize()
+                e0.record(st)
+                for _ in range(5):
+                    g.replay()
+                e1.record(st)
+                torch.cuda.synchronize()
+                graphed = e0.elapsed_time(e1) / (5 * graph_reps) * 1e3
+                del g
+                row["%s_%s" % (algo, wname)] = {"us_direct": round(direct, 2),
+                                                "us_graph": round(graphed, 2)}
+        res[name] = row
     return res
 
 
@@ -480,6 +549,8 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--ref-sample", type=int, default=262_144)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-latency", action="store_true",
+                    help="skip the small-message latency figures")
     ap.add_argument("--count", type=int, default=COUNT,
                     help="elements per rank (profiling cases only; the benchmark is 16,777,216)")
     ap.add_argument("--only", default="",

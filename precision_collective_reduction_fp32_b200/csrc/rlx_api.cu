@@ -104,6 +104,12 @@ bool vec_ok(rlx_wire wire, size_t esize, std::initializer_list<const void *> ptr
     return true;
 }
 
+// Rank buffers up to this many bytes (all ranks) take the single-launch
+// DDA-tree.
+#ifndef RLX_TREE_FUSED_MAX_BYTES
+#define RLX_TREE_FUSED_MAX_BYTES (size_t{16} << 20)
+#endif
+
 size_t tree_chunk(size_t count, int nranks) {
     const size_t blocks = (count + RLX_BLOCK - 1) / RLX_BLOCK;
     return (blocks + static_cast<size_t>(nranks) - 1) / static_cast<size_t>(nranks) * RLX_BLOCK;
@@ -240,6 +246,16 @@ rlx_status rlx_allreduce_tree(const void *send, void *recv, size_t count, size_t
         ws_scales = reinterpret_cast<float *>(ws_codes + nblk * RLX_BLOCK);
     }
     const bool vec = vec_ok(wire, es, {send, recv}, {stride});
+    // Small messages: both passes in one cooperative launch (same unit
+    // bodies, same bits); large ones: one launch per pass, whose in-order
+    // CTA runs stream HBM better.  The fused form is skipped when the device
+    // cannot launch it.
+    if (bytes <= RLX_TREE_FUSED_MAX_BYTES) {
+        const cudaError_t fe = rlx::launch_tree_fused(send, recv, count, stride, nranks, chunk,
+                                                      dtype, wire, ws_codes, ws_scales, vec, s);
+        if (fe != cudaErrorCooperativeLaunchTooLarge) return from_cuda(fe);
+        cudaGetLastError();   // clear it and fall back to two launches
+    }
     cudaError_t e = rlx::launch_tree_reduce(send, recv, count, stride, nranks, chunk, dtype, wire,
                                             ws_codes, ws_scales, vec, s);
     if (e != cudaSuccess) return from_cuda(e);

@@ -17,24 +17,11 @@
 // Units of work are numbered in memory order (segment-major) and handed out
 // in CTA-sized runs by for_each_unit, so the CTAs in flight stream one
 // compact stretch of the data.
-#include "rlx_device.cuh"
-#include "rlx_internal.h"
+#include "rlx_passes.cuh"
 
 namespace rlx {
 namespace {
 
-#ifndef RLX_UNROLL
-#define RLX_UNROLL 4
-#endif
-#ifndef RLX_J
-#define RLX_J 4
-#endif
-#ifndef RLX_JD
-#define RLX_JD 8
-#endif
-constexpr int kUnroll = RLX_UNROLL;  // 16-byte vectors per lane in flight (native copies)
-constexpr int kJ = RLX_J;            // 128-blocks in flight per warp (FP8 single-source)
-constexpr int kJd = RLX_JD;          // 128-blocks per warp when reading FP8 payloads
 #ifndef RLX_P_COPY
 #define RLX_P_COPY 1
 #endif
@@ -44,89 +31,7 @@ constexpr int kJd = RLX_JD;          // 128-blocks per warp when reading FP8 pay
 constexpr int kPc = RLX_P_COPY;      // units per warp per CTA run, native copies
 constexpr int kPg = RLX_P_GFP8;      // units per warp per CTA run, FP8 passes
 
-template <typename T> constexpr int kV = 16 / sizeof(T);
-
-// One 16-byte vector (valid elements of it) as raw bits.
-template <typename T, bool VEC>
-struct RawVec {
-    uint4 q;
-    T e[kV<T>];
-    __device__ __forceinline__ void load(const T *p, int valid) {
-        if (VEC && valid == kV<T>) {
-            q = ld_stream(reinterpret_cast<const uint4 *>(p));
-        } else {
-#pragma unroll
-            for (int k = 0; k < kV<T>; ++k)
-                if (k < valid) e[k] = p[k];
-        }
-    }
-    // default caching, for data written by the previous pass
-    __device__ __forceinline__ void load_cached(const T *p, int valid) {
-        if (VEC && valid == kV<T>) {
-            q = *reinterpret_cast<const uint4 *>(p);
-        } else {
-#pragma unroll
-            for (int k = 0; k < kV<T>; ++k)
-                if (k < valid) e[k] = p[k];
-        }
-    }
-    __device__ __forceinline__ void store(T *p, int valid) const {
-        if (VEC && valid == kV<T>) {
-            st_stream(reinterpret_cast<uint4 *>(p), q);
-        } else {
-#pragma unroll
-            for (int k = 0; k < kV<T>; ++k)
-                if (k < valid) p[k] = e[k];
-        }
-    }
-};
-
-template <typename T>
-__device__ __forceinline__ int vec_valid(size_t v, size_t nvec, size_t len) {
-    if (v >= nvec) return 0;
-    const size_t rem = len - v * kV<T>;
-    return rem < static_cast<size_t>(kV<T>) ? static_cast<int>(rem) : kV<T>;
-}
-
 // ------------------------------------------------------------------ kernels
-
-// Vectors of one unit: unit u of a segment covers vectors
-// [u*32*kUnroll, (u+1)*32*kUnroll); lane l takes u*32*kUnroll + k*32 + l, so
-// each warp store continues the previous one.
-constexpr int kWarpVecs = 32 * kUnroll;
-
-// Loads the unit's vectors of a segment of `len` elements at `src` (Full:
-// the unit lies wholly inside the segment, no bounds checks).
-template <typename T, bool VEC, bool CACHED = false, typename Full>
-__device__ __forceinline__ void load_unit(const T *src, size_t unit, size_t len, Full,
-                                          RawVec<T, VEC> (&a)[kUnroll], int (&valid)[kUnroll]) {
-    const size_t nv = (len + kV<T> - 1) / kV<T>;
-    const T *p = src + (unit * kWarpVecs + lane_id()) * kV<T>;
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-        if constexpr (Full::value) valid[u] = kV<T>;
-        else valid[u] = vec_valid<T>(unit * kWarpVecs + u * 32 + lane_id(), nv, len);
-        if (valid[u]) {
-            if (CACHED) a[u].load_cached(p + u * 32 * kV<T>, valid[u]);
-            else a[u].load(p + u * 32 * kV<T>, valid[u]);
-        }
-    }
-}
-
-template <typename T, bool VEC>
-__device__ __forceinline__ void store_unit(T *dst, size_t unit, const RawVec<T, VEC> (&a)[kUnroll],
-                                           const int (&valid)[kUnroll]) {
-    T *p = dst + (unit * kWarpVecs + lane_id()) * kV<T>;
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u)
-        if (valid[u]) a[u].store(p + u * 32 * kV<T>, valid[u]);
-}
-
-// Is unit `unit` (of kWarpVecs vectors) wholly inside a segment of len elements?
-template <typename T>
-__device__ __forceinline__ bool unit_full(size_t unit, size_t len) {
-    return (unit + 1) * kWarpVecs * kV<T> <= len;
-}
 
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
@@ -142,61 +47,25 @@ copy_kernel(const T *src, T *dst, size_t n) {
     });
 }
 
-// DDA-tree pass 2, native: unit = (chunk c, unit of it); chunk c of row c ->
-// chunk c of every other row.
+// DDA-tree pass 2, native (unit bodies in rlx_passes.cuh).
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 tree_gather_native_kernel(T *recv, size_t count, size_t stride, int n, size_t chunk,
                           FastDiv per_chunk) {
     const uint32_t units = per_chunk.d * static_cast<uint32_t>(n);
     for_each_unit<kPc>(units, [&](uint32_t g) {
-        const uint32_t c = fast_div(g, per_chunk);
-        const size_t lo = static_cast<size_t>(c) * chunk;
-        if (lo >= count) return;
-        const size_t len = count - lo < chunk ? count - lo : chunk;
-        const size_t unit = g - c * per_chunk.d;
-        with_full(unit_full<T>(unit, len), [&](auto full) {
-            RawVec<T, VEC> a[kUnroll];
-            int valid[kUnroll];
-            // the owner's chunk was just written by pass 1: default caching
-            load_unit<T, VEC, true>(recv + c * stride + lo, unit, len, full, a, valid);
-            for (int r = 0; r < n; ++r)
-                if (static_cast<uint32_t>(r) != c)
-                    store_unit<T, VEC>(recv + r * stride + lo, unit, a, valid);
-        });
+        tree_gather_native_unit<T, VEC>(g, recv, count, stride, n, chunk, per_chunk);
     });
 }
 
-// DDA-tree pass 2, FP8: unit = kJd payload blocks, dequantised into every row.
+// DDA-tree pass 2, FP8.
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 tree_gather_fp8_kernel(T *recv, size_t count, size_t stride, int n, const uint8_t *ws_codes,
                        const float *ws_scales) {
-    const size_t nblk = (count + kBlock - 1) / kBlock;
-    const uint32_t units = static_cast<uint32_t>((nblk + kJd - 1) / kJd);
-    const int e0 = lane_id() * 4;
+    const uint32_t units = static_cast<uint32_t>(tree_gather_fp8_units(count));
     for_each_unit<kPg>(units, [&](uint32_t g) {
-        const size_t b0 = static_cast<size_t>(g) * kJd;
-        with_full((b0 + kJd) * kBlock <= count, [&](auto full) {
-            constexpr bool F = decltype(full)::value;
-            const uint8_t *cp = ws_codes + b0 * kBlock + e0;
-            float y[kJd][4];
-            int valid[kJd];
-#pragma unroll
-            for (int j = 0; j < kJd; ++j) {
-                const size_t b = b0 + j;
-                valid[j] = F ? 4 : lane_valid(b * kBlock, count);
-                if (F || b < nblk) {
-                    const uint32_t codes = *reinterpret_cast<const uint32_t *>(cp + j * kBlock);
-                    dequant4(codes, ws_scales[b], y[j]);
-                }
-            }
-            for (int r = 0; r < n; ++r) {
-                T *dst = recv + r * stride + b0 * kBlock + e0;
-#pragma unroll
-                for (int j = 0; j < kJd; ++j) store4<T, VEC>(dst + j * kBlock, valid[j], y[j]);
-            }
-        });
+        tree_gather_fp8_unit<T, VEC>(g, recv, count, stride, n, ws_codes, ws_scales);
     });
 }
 
@@ -345,13 +214,13 @@ cudaError_t launch_tree_gather(void *recv, size_t count, size_t stride, int nran
     return dispatch(dtype, vec, [&]<typename T, bool VEC>() {
         T *r = static_cast<T *>(recv);
         if (wire == RLX_WIRE_NATIVE) {
-            const size_t per = copy_units<T>(chunk);
+            const size_t per = tree_gather_native_per_chunk<T>(chunk);
             if (!fits32(per)) return cudaErrorInvalidValue;
             return launch(tree_gather_native_kernel<T, VEC>, per * static_cast<size_t>(nranks),
                           kWarps * kPc, stream, r, count, stride, nranks, chunk,
                           make_fastdiv(static_cast<uint32_t>(per)));
         }
-        return launch(tree_gather_fp8_kernel<T, VEC>, block_units(count, kJd), kWarps * kPg,
+        return launch(tree_gather_fp8_kernel<T, VEC>, tree_gather_fp8_units(count), kWarps * kPg,
                       stream, r, count, stride, nranks, ws_codes, ws_scales);
     });
 }

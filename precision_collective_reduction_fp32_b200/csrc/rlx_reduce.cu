@@ -20,132 +20,10 @@
 // Units of work are numbered in memory order (chunk-major for chunked
 // passes) and handed out in CTA-sized runs by for_each_unit, so the CTAs in
 // flight stream one compact stretch of every row.
-#include "rlx_device.cuh"
-#include "rlx_internal.h"
+#include "rlx_passes.cuh"
 
 namespace rlx {
 namespace {
-
-// ------------------------------------------------------ native 16-byte vectors
-
-template <typename T> struct VecN { static constexpr int n = 16 / sizeof(T); };
-
-template <typename T, bool VEC>
-__device__ __forceinline__ void storev(T *p, int valid, const float (&v)[VecN<T>::n]) {
-    constexpr int V = VecN<T>::n;
-    if (VEC && valid == V) {
-        uint4 q;
-        if constexpr (sizeof(T) == 4) {
-            q.x = __float_as_uint(v[0]); q.y = __float_as_uint(v[1]);
-            q.z = __float_as_uint(v[2]); q.w = __float_as_uint(v[3]);
-        } else {
-            uint32_t w[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                w[k] = static_cast<uint32_t>(f32_to_bf16_bits(v[2 * k])) |
-                       (static_cast<uint32_t>(f32_to_bf16_bits(v[2 * k + 1])) << 16);
-            q = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        st_stream(reinterpret_cast<uint4 *>(p), q);
-    } else {
-#pragma unroll
-        for (int k = 0; k < V; ++k)
-            if (k < valid) Elem<T>::store(p + k, v[k]);
-    }
-}
-
-// One 16-byte vector kept as raw words (valid elements; the rest +0), so a
-// bf16 vector costs 4 registers, not 8, while all ranks are in flight.
-template <typename T, bool VEC>
-__device__ __forceinline__ uint4 loadv_raw(const T *p, int valid) {
-    constexpr int V = VecN<T>::n;
-    if (VEC && valid == V) return ld_stream(reinterpret_cast<const uint4 *>(p));
-    uint32_t w[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-    for (int k = 0; k < V; ++k) {
-        if (k < valid) {
-            if constexpr (sizeof(T) == 4)
-                w[k] = __float_as_uint(Elem<float>::load(reinterpret_cast<const float *>(p) + k));
-            else
-                w[k / 2] |= static_cast<uint32_t>(ld_stream(reinterpret_cast<const unsigned short *>(p) + k))
-                            << (16 * (k % 2));
-        }
-    }
-    return make_uint4(w[0], w[1], w[2], w[3]);
-}
-
-// Element k (compile-time) of a raw vector, widened to fp32 exactly.
-template <typename T, int K>
-__device__ __forceinline__ float raw_elem(const uint4 &q) {
-    constexpr int word = sizeof(T) == 4 ? K : K / 2;
-    const uint32_t w = word == 0 ? q.x : word == 1 ? q.y : word == 2 ? q.z : q.w;
-    if constexpr (sizeof(T) == 4) return __uint_as_float(w);
-    else return __uint_as_float(K % 2 == 0 ? w << 16 : w & 0xffff0000u);
-}
-
-template <typename T, int K = 0>
-__device__ __forceinline__ void add_raw(float (&acc)[VecN<T>::n], const uint4 &q, bool first) {
-    if constexpr (K < VecN<T>::n) {
-        const float v = raw_elem<T, K>(q);
-        acc[K] = first ? v : __fadd_rn(acc[K], v);
-        add_raw<T, K + 1>(acc, q, first);
-    }
-}
-
-// acc = x_0 + x_1 + ... + x_{n-1} (rank order) of the vector at `src` in each
-// of the n rows (row pitch `pitch` elements).  Full vectors issue all n loads
-// before the first add; a partial (tail) vector is summed rank by rank, which
-// needs few registers and keeps the kernel's register budget for the hot path.
-template <typename T, int NR, bool VEC, typename Full>
-__device__ __forceinline__ void reduce_vec(const T *src, size_t pitch, int n, int valid, Full,
-                                           float (&acc)[VecN<T>::n]) {
-    if constexpr (Full::value) {
-        uint4 x[NR];
-        const T *p = src;   // one running pointer: no per-rank address registers
-#pragma unroll
-        for (int s = 0; s < NR; ++s) {
-            if (s < n) x[s] = loadv_raw<T, VEC>(p, valid);
-            p += pitch;
-        }
-        add_raw<T>(acc, x[0], true);
-#pragma unroll
-        for (int s = 1; s < NR; ++s)
-            if (s < n) add_raw<T>(acc, x[s], false);
-    } else {
-        add_raw<T>(acc, loadv_raw<T, false>(src, valid), true);
-#pragma unroll 1
-        for (int s = 1; s < n; ++s) add_raw<T>(acc, loadv_raw<T, false>(src + s * pitch, valid), false);
-    }
-}
-
-// ---------------------------------------------------- FP8 wire, warp per block
-
-// acc = SUM_s wire(x_s) over the 128-block at `src` in each of n rows, 4
-// elements per lane (`valid` of them real; the rest +0).
-template <typename T, int NR, bool VEC>
-__device__ __forceinline__ void reduce_block_fp8(const T *src, size_t pitch, int n, int valid,
-                                                 float (&acc)[4]) {
-    float x[NR][4];
-    const int e0 = lane_id() * 4;
-#pragma unroll
-    for (int s = 0; s < NR; ++s) {
-        if (s < n) {
-            load4<T, VEC>(src + s * pitch + e0, valid, x[s]);
-        } else {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) x[s][k] = 0.0f;
-        }
-    }
-    wire_fp8_blocks<NR>(x);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) acc[k] = x[0][k];
-#pragma unroll
-    for (int s = 1; s < NR; ++s)
-        if (s < n) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) acc[k] = __fadd_rn(acc[k], x[s][k]);
-        }
-}
 
 // ------------------------------------------------------------------ kernels
 
@@ -174,18 +52,6 @@ constexpr int kPf = RLX_P_FP8;
 template <int NR> constexpr int kMinBlocksNative = NR <= 8 ? RLX_MINB_NATIVE : 1;
 template <int NR> constexpr int kMinBlocksFp8 = NR <= 8 ? RLX_MINB_FP8 : 1;
 template <int NR> constexpr int kMinBlocksFp8Flat = NR <= 8 ? RLX_MINB_FP8_FLAT : 1;
-
-// Valid elements of a vector starting at element i0 of a segment ending at
-// `hi` (V when the unit is full).
-template <int V, typename Full>
-__device__ __forceinline__ int vec_valid_in(size_t i0, size_t hi, Full) {
-    if constexpr (Full::value) {
-        return V;
-    } else {
-        if (i0 >= hi) return 0;
-        return hi - i0 < static_cast<size_t>(V) ? static_cast<int>(hi - i0) : V;
-    }
-}
 
 // DDA-flat, native: unit g = 32 consecutive 16-byte vectors (lane l: 32g + l).
 template <typename T, int NR, bool VEC>
@@ -223,51 +89,25 @@ flat_fp8_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
     });
 }
 
-// DDA-tree pass 1, native: unit = (chunk c, 32 vectors of it); chunk c -> row c.
+// DDA-tree pass 1, native (one unit body per unit, see rlx_passes.cuh).
 template <typename T, int NR, bool VEC>
 __global__ void __launch_bounds__(kThreads, kMinBlocksNative<NR>)
 tree_reduce_native_kernel(const T *send, T *recv, size_t count, size_t stride, int n,
                           size_t chunk, FastDiv per_chunk) {
-    constexpr int V = VecN<T>::n;
     const uint32_t units = per_chunk.d * static_cast<uint32_t>(n);
     for_each_unit<kPn>(units, [&](uint32_t g) {
-        const uint32_t c = fast_div(g, per_chunk);
-        const size_t lo = static_cast<size_t>(c) * chunk;
-        if (lo >= count) return;
-        const size_t hi = count - lo < chunk ? count : lo + chunk;
-        const size_t u0 = lo + static_cast<size_t>(g - c * per_chunk.d) * 32 * V;
-        const size_t i0 = u0 + static_cast<size_t>(lane_id()) * V;
-        with_full(u0 + 32 * V <= hi, [&](auto full) {
-            const int valid = vec_valid_in<V>(i0, hi, full);
-            if (valid == 0) return;
-            float acc[V];
-            reduce_vec<T, NR, VEC>(send + i0, stride, n, valid, full, acc);
-            storev<T, VEC>(recv + c * stride + i0, valid, acc);
-        });
+        tree_reduce_native_unit<T, NR, VEC>(g, send, recv, count, stride, n, chunk, per_chunk);
     });
 }
 
-// DDA-tree pass 1, FP8: unit = 128-block; reduce, then quantise the reduced
-// block again into the workspace payload (codes padded to whole blocks, one
-// scale per block).
+// DDA-tree pass 1, FP8.
 template <typename T, int NR, bool VEC>
 __global__ void __launch_bounds__(kThreads, kMinBlocksFp8<NR>)
 tree_reduce_fp8_kernel(const T *send, size_t count, size_t stride, int n,
                        uint8_t *ws_codes, float *ws_scales) {
     const uint32_t nblk = static_cast<uint32_t>((count + kBlock - 1) / kBlock);
-    const int e0 = lane_id() * 4;
     for_each_unit<kPf>(nblk, [&](uint32_t b) {
-        const size_t base = static_cast<size_t>(b) * kBlock;
-        with_full(base + kBlock <= count, [&](auto full) {
-            const int valid = decltype(full)::value ? 4 : lane_valid(base, count);
-            float acc[4];
-            reduce_block_fp8<T, NR, VEC>(send + base, stride, n, valid, acc);
-            const Scale sc = make_scale(warp_amax4(acc));
-            const uint32_t codes = quant4(acc, sc);
-            // default caching: pass 2 reads the payload back right away
-            *reinterpret_cast<uint32_t *>(ws_codes + base + e0) = codes;
-            if (lane_id() == 0) ws_scales[b] = sc.s;
-        });
+        tree_reduce_fp8_unit<T, NR, VEC>(b, send, count, stride, n, ws_codes, ws_scales);
     });
 }
 
@@ -366,7 +206,7 @@ cudaError_t launch_tree_reduce(const void *send, void *recv, size_t count, size_
     return dispatch(dtype, nranks, vec, [&]<typename T, int NR, bool VEC>() {
         const T *s = static_cast<const T *>(send);
         if (wire == RLX_WIRE_NATIVE) {
-            const size_t per = ((chunk + VecN<T>::n - 1) / VecN<T>::n + 31) / 32;
+            const size_t per = tree_reduce_native_per_chunk<T>(chunk);
             if (per >= (size_t{1} << 32)) return cudaErrorInvalidValue;
             return launch(tree_reduce_native_kernel<T, NR, VEC>,
                           per * static_cast<size_t>(nranks), kWarps * kPn, stream, s,

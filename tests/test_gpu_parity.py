@@ -204,6 +204,18 @@ def test_allreduce_inplace(algo, wire, dtype):
     assert _bits_equal(got, fn(x, wire=ORC_WIRE[wire]))
 
 
+@pytest.mark.parametrize("wire", WIRES)
+@pytest.mark.parametrize("count,inplace", [(524_288, False), (524_288, True), (524_289, False),
+                                           (600_000, True), (600_003, False)])
+def test_tree_single_and_two_launch_forms(wire, count, inplace):
+    """DDA-tree runs as one cooperative launch up to 16 MiB of rank buffers
+    (8 x 524,288 fp32 is exactly 16 MiB) and as two launches above; both
+    forms against the oracle, in place and not."""
+    x = synth.rank_buffers(4, count=count, nranks=8)
+    got = _run_allreduce("tree", x, count, count, wire, inplace=inplace)
+    assert _bits_equal(got, oracle.allreduce_tree(x, wire=ORC_WIRE[wire]))
+
+
 @pytest.mark.parametrize("algo", ["flat", "tree"])
 @pytest.mark.parametrize("wire", WIRES)
 @pytest.mark.parametrize("dtype", DTYPES)
