@@ -34,8 +34,18 @@ namespace {
 #ifndef RLX_P_FP8
 #define RLX_P_FP8 2
 #endif
+#ifndef RLX_P_FP8_FLAT
+#define RLX_P_FP8_FLAT 1
+#endif
+// FP8 tree / reduce-scatter passes with fewer blocks than this run one block
+// per warp (shorter dependent chain per warp: small-message latency), larger
+// ones RLX_P_FP8 (fewer CTA start-ups: bandwidth).
+#ifndef RLX_FP8_SMALL_BLOCKS
+#define RLX_FP8_SMALL_BLOCKS 32768
+#endif
 constexpr int kPn = RLX_P_NATIVE;
 constexpr int kPf = RLX_P_FP8;
+constexpr int kPfFlat = RLX_P_FP8_FLAT;
 
 // Resident CTAs per SM requested from the compiler (caps registers per
 // thread) for kernels with up to 8 ranks; the 16-rank forms hold twice the
@@ -78,7 +88,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocksFp8Flat<NR>)
 flat_fp8_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
     const uint32_t nblk = static_cast<uint32_t>((count + kBlock - 1) / kBlock);
     const int e0 = lane_id() * 4;
-    for_each_unit<kPf>(nblk, [&](uint32_t b) {
+    for_each_unit<kPfFlat>(nblk, [&](uint32_t b) {
         const size_t base = static_cast<size_t>(b) * kBlock;
         with_full(base + kBlock <= count, [&](auto full) {
             const int valid = decltype(full)::value ? 4 : lane_valid(base, count);
@@ -101,12 +111,12 @@ tree_reduce_native_kernel(const T *send, T *recv, size_t count, size_t stride, i
 }
 
 // DDA-tree pass 1, FP8.
-template <typename T, int NR, bool VEC>
+template <typename T, int NR, bool VEC, int P>
 __global__ void __launch_bounds__(kThreads, kMinBlocksFp8<NR>)
 tree_reduce_fp8_kernel(const T *send, size_t count, size_t stride, int n,
                        uint8_t *ws_codes, float *ws_scales) {
     const uint32_t nblk = static_cast<uint32_t>((count + kBlock - 1) / kBlock);
-    for_each_unit<kPf>(nblk, [&](uint32_t b) {
+    for_each_unit<P>(nblk, [&](uint32_t b) {
         tree_reduce_fp8_unit<T, NR, VEC>(b, send, count, stride, n, ws_codes, ws_scales);
     });
 }
@@ -134,13 +144,13 @@ rs_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t 
 
 // ReduceScatter, FP8: unit = (destination rank r, 128-block of chunk r);
 // blocks anchored at the chunk start r*m.
-template <typename T, int NR, bool VEC>
+template <typename T, int NR, bool VEC, int P>
 __global__ void __launch_bounds__(kThreads, kMinBlocksFp8<NR>)
 rs_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n,
               FastDiv per_chunk) {
     const uint32_t units = per_chunk.d * static_cast<uint32_t>(n);
     const int e0 = lane_id() * 4;
-    for_each_unit<kPf>(units, [&](uint32_t g) {
+    for_each_unit<P>(units, [&](uint32_t g) {
         const uint32_t r = fast_div(g, per_chunk);
         const size_t j0 = static_cast<size_t>(g - r * per_chunk.d) * kBlock;
         with_full(j0 + kBlock <= m, [&](auto full) {
@@ -194,7 +204,7 @@ cudaError_t launch_allreduce_flat(const void *send, void *recv, size_t count, si
                           count, stride, nranks);
         }
         const size_t nblk = (count + kBlock - 1) / kBlock;
-        return launch(flat_fp8_kernel<T, NR, VEC>, nblk, kWarps * kPf, stream, s, r, count,
+        return launch(flat_fp8_kernel<T, NR, VEC>, nblk, kWarps * kPfFlat, stream, s, r, count,
                       stride, nranks);
     });
 }
@@ -214,8 +224,11 @@ cudaError_t launch_tree_reduce(const void *send, void *recv, size_t count, size_
                           make_fastdiv(static_cast<uint32_t>(per)));
         }
         const size_t nblk = (count + kBlock - 1) / kBlock;
-        return launch(tree_reduce_fp8_kernel<T, NR, VEC>, nblk, kWarps * kPf, stream, s, count,
-                      stride, nranks, ws_codes, ws_scales);
+        if (nblk < RLX_FP8_SMALL_BLOCKS)
+            return launch(tree_reduce_fp8_kernel<T, NR, VEC, 1>, nblk, kWarps, stream, s, count,
+                          stride, nranks, ws_codes, ws_scales);
+        return launch(tree_reduce_fp8_kernel<T, NR, VEC, kPf>, nblk, kWarps * kPf, stream, s,
+                      count, stride, nranks, ws_codes, ws_scales);
     });
 }
 
@@ -233,8 +246,11 @@ cudaError_t launch_reduce_scatter(const void *send, size_t send_stride, void *re
         if (wire == RLX_WIRE_NATIVE)
             return launch(rs_native_kernel<T, NR, VEC>, per * nn, kWarps * kPn, stream, s,
                           send_stride, r, recv_stride, m, nranks, fd);
-        return launch(rs_fp8_kernel<T, NR, VEC>, per * nn, kWarps * kPf, stream, s, send_stride,
-                      r, recv_stride, m, nranks, fd);
+        if (per * nn < RLX_FP8_SMALL_BLOCKS)
+            return launch(rs_fp8_kernel<T, NR, VEC, 1>, per * nn, kWarps, stream, s, send_stride,
+                          r, recv_stride, m, nranks, fd);
+        return launch(rs_fp8_kernel<T, NR, VEC, kPf>, per * nn, kWarps * kPf, stream, s,
+                      send_stride, r, recv_stride, m, nranks, fd);
     });
 }
 
