@@ -50,7 +50,8 @@
  *     alignment (16 B rows and chunks) selects the vectorised kernels;
  *     anything else runs element-wise kernels with the same results.
  *   - nranks is 1..RLX_MAX_RANKS.  Row strides are in elements.
- *   - Size products that overflow size_t are rejected (RLX_ERR_INVALID_ARG).
+ *   - Size products that overflow size_t, and calls over RLX_MAX_ELEMENTS
+ *     elements (all ranks together), are rejected (RLX_ERR_INVALID_ARG).
  *   - FP8-wire inputs must be finite; non-finite inputs give unspecified codes.
  */
 #ifndef RLX_H
@@ -71,6 +72,9 @@ extern "C" {
 
 #define RLX_BLOCK 128     /* elements per FP8 scale block           */
 #define RLX_MAX_RANKS 16  /* largest simulated rank count supported */
+/* Largest element count of one call, all ranks (rows) together: 2^36, more
+ * than any B200 holds; larger requests return RLX_ERR_INVALID_ARG. */
+#define RLX_MAX_ELEMENTS ((size_t)1 << 36)
 
 typedef enum {
     RLX_OK = 0,

@@ -65,6 +65,7 @@ namespace {
 size_t elem_size(rlx_dtype d) { return d == RLX_BF16 ? 2 : 4; }
 
 bool dtype_ok(rlx_dtype d) { return d == RLX_F32 || d == RLX_BF16; }
+
 bool wire_ok(rlx_wire w) { return w == RLX_WIRE_NATIVE || w == RLX_WIRE_FP8_E4M3; }
 bool ranks_ok(int n) { return n >= 1 && n <= RLX_MAX_RANKS; }
 
@@ -74,6 +75,13 @@ bool mul(size_t a, size_t b, size_t *out) {
     return true;
 }
 
+// Every kernel numbers its units of work with 32 bits; up to RLX_MAX_ELEMENTS
+// elements per call (all ranks together) the largest unit count stays far
+// below 2^32.  No B200 holds more.
+bool size_ok(size_t rows, size_t n) {
+    size_t total = 0;
+    return mul(rows, n, &total) && total <= RLX_MAX_ELEMENTS;
+}
 // Bytes spanned by `rows` rows of `len` elements at pitch `stride` elements.
 bool extent(size_t rows, size_t stride, size_t len, size_t esize, size_t *bytes) {
     size_t a, b;
@@ -163,7 +171,7 @@ rlx_status rlx_quantize_fp8(const void *x, rlx_dtype dtype, size_t rows, size_t 
                             size_t stride, uint8_t *codes, float *scales, void *stream) {
     if (!dtype_ok(dtype) || stride < n) return RLX_ERR_INVALID_ARG;
     if (rows == 0 || n == 0) return RLX_OK;
-    if (!x || !codes || !scales) return RLX_ERR_INVALID_ARG;
+    if (!x || !codes || !scales || !size_ok(rows, n)) return RLX_ERR_INVALID_ARG;
     const size_t es = elem_size(dtype);
     size_t xb, cb, sb, nbr = (n + RLX_BLOCK - 1) / RLX_BLOCK;
     if (!extent(rows, stride, n, es, &xb) || !extent(rows, stride, n, 1, &cb) ||
@@ -182,7 +190,7 @@ rlx_status rlx_dequantize_fp8(const uint8_t *codes, const float *scales, size_t 
                               void *stream) {
     if (!dtype_ok(dtype) || stride < n) return RLX_ERR_INVALID_ARG;
     if (rows == 0 || n == 0) return RLX_OK;
-    if (!y || !codes || !scales) return RLX_ERR_INVALID_ARG;
+    if (!y || !codes || !scales || !size_ok(rows, n)) return RLX_ERR_INVALID_ARG;
     const size_t es = elem_size(dtype);
     size_t yb, cb, sb, nbr = (n + RLX_BLOCK - 1) / RLX_BLOCK;
     if (!extent(rows, stride, n, es, &yb) || !extent(rows, stride, n, 1, &cb) ||
@@ -204,7 +212,7 @@ static rlx_status check_allreduce(const void *send, void *recv, size_t count, si
         return RLX_ERR_INVALID_ARG;
     if (op != RLX_SUM) return RLX_ERR_UNSUPPORTED;
     if (count == 0) { *bytes = 0; return RLX_OK; }
-    if (!send || !recv) return RLX_ERR_INVALID_ARG;
+    if (!send || !recv || !size_ok(static_cast<size_t>(nranks), count)) return RLX_ERR_INVALID_ARG;
     const size_t es = elem_size(dtype);
     if (!extent(static_cast<size_t>(nranks), stride, count, es, bytes)) return RLX_ERR_INVALID_ARG;
     if (!aligned(send, es) || !aligned(recv, es)) return RLX_ERR_ALIGNMENT;
@@ -284,6 +292,7 @@ static rlx_status check_chunked(const void *send, size_t sstride, size_t slen, v
     const size_t es = elem_size(dtype);
     if (slen == 0 || rlen == 0 || sstride < slen || rstride < rlen)
         return RLX_ERR_INVALID_ARG;
+    if (!size_ok(static_cast<size_t>(nranks), slen > rlen ? slen : rlen)) return RLX_ERR_INVALID_ARG;
     if (!send || !recv) return RLX_ERR_INVALID_ARG;
     if (!extent(static_cast<size_t>(nranks), sstride, slen, es, &sb) ||
         !extent(static_cast<size_t>(nranks), rstride, rlen, es, &rb))

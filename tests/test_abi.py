@@ -127,6 +127,20 @@ def test_quant_validation(L):
     assert d(A, A + Z + 1, 2, 100, 100, A + 2 * Z, F32) == B.RLX_ERR_ALIGNMENT
 
 
+def test_element_limit(L):
+    """2^36 elements per call (all ranks) at most; one more is rejected before
+    any CUDA call (the pointers here are never touched)."""
+    big = (1 << 36) // 8 + 1
+    assert _st("rlx_allreduce_flat", A, A + (1 << 40), big, big, 8, F32, NAT, SUM, None) == \
+        B.RLX_ERR_INVALID_ARG
+    assert _st("rlx_allreduce_tree", A, A + (1 << 40), big, big, 8, F32, FP8, SUM, None, 0, None) == \
+        B.RLX_ERR_INVALID_ARG
+    assert _st("rlx_alltoall", A, 8 * big, A + (1 << 42), 8 * big, big, 8, F32, NAT, None) == \
+        B.RLX_ERR_INVALID_ARG
+    assert _st("rlx_quantize_fp8", A, F32, 8, big, big, A + (1 << 40), A + (1 << 41), None) == \
+        B.RLX_ERR_INVALID_ARG
+
+
 def test_no_cuda_error_recorded(L):
     """None of the rejected calls above reached CUDA."""
     assert B.rlx_last_cuda_error() == 0
