@@ -430,11 +430,7 @@ def small_message_latency(dev, reps: int = 200, graph_reps: int = 50) -> dict:
                                                    B.RLX_WIRE_FP8_E4M3), 16),
                          dtype=torch.uint8, device=dev)
         row = {}
-        for algo in ("flat", "tree", "tree1"):   # tree1: the opt-in single-launch DDA-tree
-            if algo == "tree1":
-                os.environ["RLX_TREE_FUSED_MAX_BYTES"] = str(1 << 40)
-            else:
-                os.environ.pop("RLX_TREE_FUSED_MAX_BYTES", None)
+        for algo in ("flat", "tree"):
             for wname, wire in (("native", B.RLX_WIRE_NATIVE), ("fp8", B.RLX_WIRE_FP8_E4M3)):
                 def call(stream_ptr):
                     if algo == "flat":
@@ -473,7 +469,6 @@ def small_message_latency(dev, reps: int = 200, graph_reps: int = 50) -> dict:
                 del g
                 row["%s_%s" % (algo, wname)] = {"us_direct": round(direct, 2),
                                                 "us_graph": round(graphed, 2)}
-        os.environ.pop("RLX_TREE_FUSED_MAX_BYTES", None)
         res[name] = row
     return res
 

@@ -3,7 +3,6 @@
 // Nothing here touches the data; every arithmetic step runs in the kernels.
 #include <climits>
 #include <cstdint>
-#include <cstdlib>
 #include <map>
 #include <mutex>
 #include <utility>
@@ -111,22 +110,6 @@ bool vec_ok(rlx_wire wire, size_t esize, std::initializer_list<const void *> ptr
     for (size_t o : offsets)
         if (o % elems != 0) return false;
     return true;
-}
-
-// Rank buffers (all ranks together) up to this many bytes take the
-// single-launch DDA-tree; 0 = never.  Off by default: on B200 a cooperative
-// launch cannot start while the previous kernel drains, which costs more GPU
-// time than the saved launch (measured: 5.7 vs 5.3 us for 8 x 512 KiB bf16
-// replayed from a CUDA graph); it pays off only when each launch carries a
-// host-side cost (7.2 vs 9.2 us launched one by one from Python).  The
-// environment variable RLX_TREE_FUSED_MAX_BYTES, read at every call,
-// overrides the default.
-size_t tree_fused_max_bytes() {
-    const char *v = std::getenv("RLX_TREE_FUSED_MAX_BYTES");
-    if (v == nullptr || *v == '\0') return 0;
-    char *end = nullptr;
-    const unsigned long long b = std::strtoull(v, &end, 10);
-    return (end != nullptr && *end == '\0') ? static_cast<size_t>(b) : 0;
 }
 
 size_t tree_chunk(size_t count, int nranks) {
@@ -265,16 +248,6 @@ rlx_status rlx_allreduce_tree(const void *send, void *recv, size_t count, size_t
         ws_scales = reinterpret_cast<float *>(ws_codes + nblk * RLX_BLOCK);
     }
     const bool vec = vec_ok(wire, es, {send, recv}, {stride});
-    // Small messages: both passes in one cooperative launch (same unit
-    // bodies, same bits); large ones: one launch per pass, whose in-order
-    // CTA runs stream HBM better.  The fused form is skipped when the device
-    // cannot launch it.
-    if (bytes <= tree_fused_max_bytes()) {
-        const cudaError_t fe = rlx::launch_tree_fused(send, recv, count, stride, nranks, chunk,
-                                                      dtype, wire, ws_codes, ws_scales, vec, s);
-        if (fe != cudaErrorCooperativeLaunchTooLarge) return from_cuda(fe);
-        cudaGetLastError();   // clear it and fall back to two launches
-    }
     cudaError_t e = rlx::launch_tree_reduce(send, recv, count, stride, nranks, chunk, dtype, wire,
                                             ws_codes, ws_scales, vec, s);
     if (e != cudaSuccess) return from_cuda(e);

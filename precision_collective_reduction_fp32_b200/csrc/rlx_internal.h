@@ -35,14 +35,6 @@ cudaError_t launch_tree_reduce(const void *send, void *recv, size_t count, size_
                                uint8_t *ws_codes, float *ws_scales, bool vec,
                                cudaStream_t stream);
 
-// DDA-tree, both passes in one cooperative launch (small messages).  Fails
-// with cudaErrorCooperativeLaunchTooLarge when cooperative launches are not
-// available; nothing runs then.
-cudaError_t launch_tree_fused(const void *send, void *recv, size_t count, size_t stride,
-                              int nranks, size_t chunk, rlx_dtype dtype, rlx_wire wire,
-                              uint8_t *ws_codes, float *ws_scales, bool vec,
-                              cudaStream_t stream);
-
 // DDA-tree pass 2 (all-gather).
 cudaError_t launch_tree_gather(void *recv, size_t count, size_t stride, int nranks,
                                size_t chunk, rlx_dtype dtype, rlx_wire wire,

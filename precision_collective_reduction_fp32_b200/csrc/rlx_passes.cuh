@@ -1,6 +1,5 @@
 // rlx_passes.cuh -- per-unit bodies of the streaming passes, shared by the
-// kernels that run one pass per launch (rlx_reduce.cu, rlx_gather.cu) and
-// the single-launch DDA-tree (rlx_tree_fused.cu): native 16-byte vector
+// kernels of rlx_reduce.cu and rlx_gather.cu: native 16-byte vector
 // reductions and copies, the FP8-wire block reduction, and one unit of each
 // DDA-tree pass.
 #pragma once

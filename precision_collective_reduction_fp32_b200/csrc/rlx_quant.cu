@@ -26,13 +26,18 @@ namespace {
 #ifndef RLX_P_DQ
 #define RLX_P_DQ 1
 #endif
+// Resident CTAs per SM requested from the compiler for the quantiser
+// (0: no request).
+#ifndef RLX_MINB_Q
+#define RLX_MINB_Q 0
+#endif
 constexpr int kJq = RLX_JQ;    // blocks in flight per warp, quantise
 constexpr int kJd = RLX_JDQ;   // blocks in flight per warp, dequantise
 constexpr int kPq = RLX_P_Q;   // units per warp per CTA run, quantise
 constexpr int kPdq = RLX_P_DQ; // units per warp per CTA run, dequantise
 
 template <typename T, bool VEC>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, RLX_MINB_Q)
 quantize_kernel(const T *x, size_t rows, size_t n, size_t stride, uint8_t *codes,
                 float *scales, FastDiv per_row) {
     const size_t nbr = (n + kBlock - 1) / kBlock;

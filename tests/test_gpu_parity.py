@@ -205,16 +205,11 @@ def test_allreduce_inplace(algo, wire, dtype):
 
 
 @pytest.mark.parametrize("wire", WIRES)
-@pytest.mark.parametrize("dtype", DTYPES)
-@pytest.mark.parametrize("count,inplace", [(1, False), (200, False), (3000, True),
-                                           (131_075, False), (524_288, True), (524_289, False)])
-def test_tree_single_launch_form(monkeypatch, wire, dtype, count, inplace):
-    """The opt-in single-launch DDA-tree (RLX_TREE_FUSED_MAX_BYTES): rank
-    buffers up to the limit run pass 1, a grid barrier and pass 2 in one
-    cooperative launch; above it, two launches.  8 x 524,288 fp32 is exactly
-    16 MiB.  Both forms against the oracle, in place and not."""
-    monkeypatch.setenv("RLX_TREE_FUSED_MAX_BYTES", str(16 << 20))
-    x = synth.rank_buffers(4, count=count, nranks=8, dtype=dtype)
+@pytest.mark.parametrize("count,inplace", [(524_288, True), (600_003, False)])
+def test_tree_in_place_mid_size(wire, count, inplace):
+    """DDA-tree at a few MiB per rank, in place and not: pass 2 re-reads rows
+    pass 1 streamed as input and just rewrote (read through L2 only)."""
+    x = synth.rank_buffers(4, count=count, nranks=8)
     got = _run_allreduce("tree", x, count, count, wire, inplace=inplace)
     assert _bits_equal(got, oracle.allreduce_tree(x, wire=ORC_WIRE[wire]))
 
