@@ -205,13 +205,54 @@ __device__ __forceinline__ float quotient_rn(float x, float s, float y) {
     return __fmaf_rn(-r, y, q);
 }
 
+// Blackwell executes two fp32 lanes per instruction (add/mul/fma .f32x2);
+// each lane rounds exactly like the scalar instruction, so the packed forms
+// below give the same bits with half the instructions.  RLX_PACKED_F32X2=0
+// selects the scalar forms.
+#ifndef RLX_PACKED_F32X2
+#define RLX_PACKED_F32X2 1
+#endif
+
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+
+// quotient_rn on two values sharing (s, y): the same steps, two lanes each.
+__device__ __forceinline__ float2 quotient_rn2(float2 x, float s, float y) {
+#if RLX_PACKED_F32X2
+    const float2 s2 = f2(s, s), y2 = f2(y, y), ny2 = f2(-y, -y), nx = f2(-x.x, -x.y);
+    float2 q = __fmul2_rn(x, y2);
+    float2 r = __ffma2_rn(s2, q, nx);   // s*q - x
+    q = __ffma2_rn(r, ny2, q);          // q - r*y
+    r = __ffma2_rn(s2, q, nx);
+    return __ffma2_rn(r, ny2, q);
+#else
+    return f2(quotient_rn(x.x, s, y), quotient_rn(x.y, s, y));
+#endif
+}
+
+__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
+#if RLX_PACKED_F32X2
+    return __fmul2_rn(a, b);
+#else
+    return f2(__fmul_rn(a.x, b.x), __fmul_rn(a.y, b.y));
+#endif
+}
+
+__device__ __forceinline__ float2 add2_rn(float2 a, float2 b) {
+#if RLX_PACKED_F32X2
+    return __fadd2_rn(a, b);
+#else
+    return f2(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y));
+#endif
+}
+
 // Quantise 4 values of a block with scale sc: code = e4m3_rne_sat(fl32(v/s));
 // s == 0 gives signed zeros.  sc.y == 0 selects the IEEE division.
 __device__ __forceinline__ uint32_t quant4(const float (&v)[4], Scale sc) {
     float q[4];
     if (sc.y != 0.0f) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) q[k] = quotient_rn(v[k], sc.s, sc.y);
+        const float2 a = quotient_rn2(f2(v[0], v[1]), sc.s, sc.y);
+        const float2 b = quotient_rn2(f2(v[2], v[3]), sc.s, sc.y);
+        q[0] = a.x; q[1] = a.y; q[2] = b.x; q[3] = b.y;
     } else if (sc.s == 0.0f) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) q[k] = __fmul_rn(v[k], 0.0f);  // +-0 with v's sign
@@ -224,12 +265,9 @@ __device__ __forceinline__ uint32_t quant4(const float (&v)[4], Scale sc) {
 
 // Dequantise 4 packed codes with scale s: fl32(e4m3(code) * s).
 __device__ __forceinline__ void dequant4(uint32_t codes, float s, float (&y)[4]) {
-    const float2 a = e4m3x2_to_f32(codes & 0xffffu);
-    const float2 b = e4m3x2_to_f32(codes >> 16);
-    y[0] = __fmul_rn(a.x, s);
-    y[1] = __fmul_rn(a.y, s);
-    y[2] = __fmul_rn(b.x, s);
-    y[3] = __fmul_rn(b.y, s);
+    const float2 a = mul2_rn(e4m3x2_to_f32(codes & 0xffffu), f2(s, s));
+    const float2 b = mul2_rn(e4m3x2_to_f32(codes >> 16), f2(s, s));
+    y[0] = a.x; y[1] = a.y; y[2] = b.x; y[3] = b.y;
 }
 
 // What a receiver holds after K 128-blocks crossed the FP8 wire.  The warp

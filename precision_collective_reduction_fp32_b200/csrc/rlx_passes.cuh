@@ -68,10 +68,17 @@ __device__ __forceinline__ float raw_elem(const uint4 &q) {
 
 template <typename T, int K = 0>
 __device__ __forceinline__ void add_raw(float (&acc)[VecN<T>::n], const uint4 &q, bool first) {
-    if constexpr (K < VecN<T>::n) {
-        const float v = raw_elem<T, K>(q);
-        acc[K] = first ? v : __fadd_rn(acc[K], v);
-        add_raw<T, K + 1>(acc, q, first);
+    if constexpr (K < VecN<T>::n) {   // two elements per step (packed add)
+        const float2 v = f2(raw_elem<T, K>(q), raw_elem<T, K + 1>(q));
+        if (first) {
+            acc[K] = v.x;
+            acc[K + 1] = v.y;
+        } else {
+            const float2 s = add2_rn(f2(acc[K], acc[K + 1]), v);
+            acc[K] = s.x;
+            acc[K + 1] = s.y;
+        }
+        add_raw<T, K + 2>(acc, q, first);
     }
 }
 
@@ -120,14 +127,14 @@ __device__ __forceinline__ void reduce_block_fp8(const T *src, size_t pitch, int
         }
     }
     wire_fp8_blocks<NR>(x);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) acc[k] = x[0][k];
+    float2 a01 = f2(x[0][0], x[0][1]), a23 = f2(x[0][2], x[0][3]);
 #pragma unroll
     for (int s = 1; s < NR; ++s)
         if (s < n) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) acc[k] = __fadd_rn(acc[k], x[s][k]);
+            a01 = add2_rn(a01, f2(x[s][0], x[s][1]));
+            a23 = add2_rn(a23, f2(x[s][2], x[s][3]));
         }
+    acc[0] = a01.x; acc[1] = a01.y; acc[2] = a23.x; acc[3] = a23.y;
 }
 
 // Valid elements of a vector starting at element i0 of a segment ending at
