@@ -11,9 +11,10 @@
 // On the native wire these passes move bytes only (16-byte vectors, no
 // conversion), so results are bit copies; a warp moves kUnroll x 512
 // contiguous bytes per step (lane l takes vectors l, l+32, ...), so each of
-// its stores to a destination row continues the previous one.  On the FP8 wire a warp handles kJ consecutive 128-element blocks
-// at once (4 elements per lane per block): it reads them, applies
-// dequantise(quantise(.)) in registers and writes every destination.
+// its stores to a destination row continues the previous one.  On the FP8
+// wire a warp handles kJ consecutive 128-element blocks at once (4 elements
+// per lane per block): it reads them, applies dequantise(quantise(.)) in
+// registers and writes every destination.
 // Units of work are numbered in memory order (segment-major) and handed out
 // in CTA-sized runs by for_each_unit, so the CTAs in flight stream one
 // compact stretch of the data.

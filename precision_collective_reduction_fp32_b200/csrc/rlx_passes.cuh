@@ -166,7 +166,6 @@ constexpr int kJd = RLX_JD;          // 128-blocks per warp when reading FP8 pay
 
 template <typename T> constexpr int kV = 16 / sizeof(T);
 
-// One 16-byte vector (valid elements of it) as raw bits.
 // One element read through L2 only.
 template <typename T>
 __device__ __forceinline__ T load_l2(const T *p) {
@@ -178,6 +177,7 @@ __device__ __forceinline__ T load_l2(const T *p) {
     }
 }
 
+// One 16-byte vector (valid elements of it) as raw bits.
 template <typename T, bool VEC>
 struct RawVec {
     uint4 q;
@@ -193,7 +193,7 @@ struct RawVec {
     }
     // for data the previous pass just wrote (possibly from another SM): read
     // through L2 only (ld.global.cg), never from a possibly stale L1 line
-    __device__ __forceinline__ void load_cached(const T *p, int valid) {
+    __device__ __forceinline__ void load_through_l2(const T *p, int valid) {
         if (VEC && valid == kV<T>) {
             q = __ldcg(reinterpret_cast<const uint4 *>(p));
         } else {
@@ -227,7 +227,7 @@ constexpr int kWarpVecs = 32 * kUnroll;
 
 // Loads the unit's vectors of a segment of `len` elements at `src` (Full:
 // the unit lies wholly inside the segment, no bounds checks).
-template <typename T, bool VEC, bool CACHED = false, typename Full>
+template <typename T, bool VEC, bool THROUGH_L2 = false, typename Full>
 __device__ __forceinline__ void load_unit(const T *src, size_t unit, size_t len, Full,
                                           RawVec<T, VEC> (&a)[kUnroll], int (&valid)[kUnroll]) {
     const size_t nv = (len + kV<T> - 1) / kV<T>;
@@ -237,7 +237,7 @@ __device__ __forceinline__ void load_unit(const T *src, size_t unit, size_t len,
         if constexpr (Full::value) valid[u] = kV<T>;
         else valid[u] = vec_valid<T>(unit * kWarpVecs + u * 32 + lane_id(), nv, len);
         if (valid[u]) {
-            if (CACHED) a[u].load_cached(p + u * 32 * kV<T>, valid[u]);
+            if (THROUGH_L2) a[u].load_through_l2(p + u * 32 * kV<T>, valid[u]);
             else a[u].load(p + u * 32 * kV<T>, valid[u]);
         }
     }
@@ -315,7 +315,7 @@ __device__ __forceinline__ void tree_gather_native_unit(uint32_t g, T *recv, siz
     with_full(unit_full<T>(unit, len), [&](auto full) {
         RawVec<T, VEC> a[kUnroll];
         int valid[kUnroll];
-        // the owner's chunk was just written by pass 1: default caching
+        // the owner's chunk was just written by pass 1: read it through L2
         load_unit<T, VEC, true>(recv + c * stride + lo, unit, len, full, a, valid);
         for (int r = 0; r < n; ++r)
             if (static_cast<uint32_t>(r) != c)
