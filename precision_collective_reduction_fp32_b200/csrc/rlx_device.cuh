@@ -320,9 +320,21 @@ __host__ __device__ __forceinline__ uint32_t fast_div(uint32_t n, const FastDiv 
 // are started in index order, so the CTAs resident at any moment work on one
 // compact stretch of the data, which keeps few DRAM pages open.  f(g) is
 // called with the same g by all 32 lanes.
+// Programmatic dependent launch: the kernels are launched so that the next
+// kernel on the stream may be scheduled while this one finishes its last
+// wave.  Before its first memory access every kernel waits until the grids it
+// depends on have completed and their writes are visible (griddepcontrol.wait
+// returns at once when there is no such grid), and it lets its own dependents
+// be scheduled as soon as all of its CTAs are running.
+__device__ __forceinline__ void pdl_begin() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
+}
+
 template <int P, typename F>
 __device__ __forceinline__ void for_each_unit(uint32_t total, F &&f) {
     constexpr uint32_t W = 256 / 32;   // rlx kernels run 256-thread CTAs
+    pdl_begin();                       // every kernel's first memory access comes after this
     const uint32_t w = threadIdx.x >> 5;
     const size_t span = static_cast<size_t>(W) * P;
     for (size_t base = blockIdx.x * span; base < total; base += gridDim.x * span) {

@@ -185,8 +185,7 @@ cudaError_t launch(K kernel, size_t units, size_t units_per_cta, cudaStream_t st
                    Args... args) {
     const dim3 grid = grid_for(reinterpret_cast<const void *>(kernel), units, units_per_cta);
     if (grid.x == 0) return cudaErrorInvalidValue;
-    kernel<<<grid, kThreads, 0, stream>>>(args...);
-    return cudaGetLastError();
+    return launch_kernel(kernel, grid, stream, args...);
 }
 
 constexpr size_t kWarps = kThreads / 32;

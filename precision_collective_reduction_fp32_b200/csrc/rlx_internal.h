@@ -20,6 +20,29 @@ constexpr int kThreads = 256;  // threads per CTA for every kernel
 // an empty grid.
 dim3 grid_for(const void *kernel, size_t units, size_t units_per_cta);
 
+// Launches kernel<<<grid, kThreads, 0, stream>>>(args...) allowing
+// programmatic dependent launch (RLX_PDL=1, default): the kernel may be
+// scheduled while the previous kernel on the stream finishes; every rlx
+// kernel waits for it (griddepcontrol.wait) before touching memory.
+#ifndef RLX_PDL
+#define RLX_PDL 1
+#endif
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, cudaStream_t stream,
+                          Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = RLX_PDL;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // Records a CUDA failure for rlx_last_cuda_error() of the calling thread.
 void record_cuda_error(cudaError_t e);
 

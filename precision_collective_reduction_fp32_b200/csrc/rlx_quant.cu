@@ -146,8 +146,7 @@ cudaError_t launch_rows(K kernel, size_t rows, size_t n, size_t blocks_per_unit,
     const dim3 grid = grid_for(reinterpret_cast<const void *>(kernel), per * rows,
                                kWarps * units_per_warp);
     if (grid.x == 0) return cudaErrorInvalidValue;
-    kernel<<<grid, kThreads, 0, stream>>>(args..., make_fastdiv(static_cast<uint32_t>(per)));
-    return cudaGetLastError();
+    return launch_kernel(kernel, grid, stream, args..., make_fastdiv(static_cast<uint32_t>(per)));
 }
 
 }  // namespace
