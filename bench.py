@@ -215,36 +215,43 @@ class Step:
         t = lambda *s, dt=torch.float32: torch.empty(*s, dtype=dt, device=device)
         self.x = t((n, self.pitch))
         self.x[:, :c].copy_(torch.from_numpy(x_host))
-        self.out = t((n, self.pitch))
-        self.y = t((n, self.pitch))
+        # two of each output, alternated so that no operation writes the
+        # buffer its predecessor has just written (dirty L2 lines of one
+        # operation are never overwritten by the next)
+        self.out1, self.out2 = t((n, self.pitch)), t((n, self.pitch))
+        self.y1, self.y2 = t((n, self.pitch)), t((n, self.pitch))
+        self.out = self.out2                       # holds the FP8 tree allreduce result
         self.codes = t((n, self.pitch), dt=torch.uint8)
         self.scales = t((n, (c + BLOCK - 1) // BLOCK))
-        self.rs = t((n, self.mpitch))
+        self.rs1, self.rs2 = t((n, self.mpitch)), t((n, self.mpitch))
         self.ws_bytes = B.rlx_workspace_bytes(B.RLX_COLL_ALLREDUCE_TREE, c, n, B.RLX_F32,
                                               B.RLX_WIRE_FP8_E4M3)
         self.ws = t((self.ws_bytes,), dt=torch.uint8)
 
     def ops(self, stream):
         B, n, c, m, p, mp = self.B, self.n, self.c, self.m, self.pitch, self.mpitch
-        x, out, y, rs = self.x.data_ptr(), self.out.data_ptr(), self.y.data_ptr(), self.rs.data_ptr()
+        x = self.x.data_ptr()
+        o1, o2 = self.out1.data_ptr(), self.out2.data_ptr()
+        y1, y2 = self.y1.data_ptr(), self.y2.data_ptr()
+        r1, r2 = self.rs1.data_ptr(), self.rs2.data_ptr()
         F, NAT, FP8 = B.RLX_F32, B.RLX_WIRE_NATIVE, B.RLX_WIRE_FP8_E4M3
         return [
             ("quantize_fp8", lambda: B.rlx_quantize_fp8(x, F, n, c, p, self.codes.data_ptr(),
                                                         self.scales.data_ptr(), stream)),
             ("dequantize_fp8", lambda: B.rlx_dequantize_fp8(self.codes.data_ptr(), self.scales.data_ptr(),
-                                                            n, c, p, y, F, stream)),
-            ("allreduce_flat_native", lambda: B.rlx_allreduce_flat(x, out, c, p, n, F, NAT, B.RLX_SUM, stream)),
-            ("allreduce_flat_fp8", lambda: B.rlx_allreduce_flat(x, out, c, p, n, F, FP8, B.RLX_SUM, stream)),
-            ("allreduce_tree_native", lambda: B.rlx_allreduce_tree(x, out, c, p, n, F, NAT, B.RLX_SUM,
+                                                            n, c, p, y2, F, stream)),
+            ("allreduce_flat_native", lambda: B.rlx_allreduce_flat(x, o1, c, p, n, F, NAT, B.RLX_SUM, stream)),
+            ("allreduce_flat_fp8", lambda: B.rlx_allreduce_flat(x, o2, c, p, n, F, FP8, B.RLX_SUM, stream)),
+            ("allreduce_tree_native", lambda: B.rlx_allreduce_tree(x, o1, c, p, n, F, NAT, B.RLX_SUM,
                                                                    None, 0, stream)),
-            ("allreduce_tree_fp8", lambda: B.rlx_allreduce_tree(x, out, c, p, n, F, FP8, B.RLX_SUM,
+            ("allreduce_tree_fp8", lambda: B.rlx_allreduce_tree(x, o2, c, p, n, F, FP8, B.RLX_SUM,
                                                                 self.ws.data_ptr(), self.ws_bytes, stream)),
-            ("reduce_scatter_native", lambda: B.rlx_reduce_scatter(x, p, rs, mp, m, n, F, NAT, B.RLX_SUM, stream)),
-            ("reduce_scatter_fp8", lambda: B.rlx_reduce_scatter(x, p, rs, mp, m, n, F, FP8, B.RLX_SUM, stream)),
-            ("all_gather_native", lambda: B.rlx_all_gather(rs, mp, y, p, m, n, F, NAT, stream)),
-            ("all_gather_fp8", lambda: B.rlx_all_gather(rs, mp, y, p, m, n, F, FP8, stream)),
-            ("alltoall_native", lambda: B.rlx_alltoall(x, p, y, p, m, n, F, NAT, stream)),
-            ("alltoall_fp8", lambda: B.rlx_alltoall(x, p, y, p, m, n, F, FP8, stream)),
+            ("reduce_scatter_native", lambda: B.rlx_reduce_scatter(x, p, r1, mp, m, n, F, NAT, B.RLX_SUM, stream)),
+            ("reduce_scatter_fp8", lambda: B.rlx_reduce_scatter(x, p, r2, mp, m, n, F, FP8, B.RLX_SUM, stream)),
+            ("all_gather_native", lambda: B.rlx_all_gather(r1, mp, y1, p, m, n, F, NAT, stream)),
+            ("all_gather_fp8", lambda: B.rlx_all_gather(r2, mp, y2, p, m, n, F, FP8, stream)),
+            ("alltoall_native", lambda: B.rlx_alltoall(x, p, y1, p, m, n, F, NAT, stream)),
+            ("alltoall_fp8", lambda: B.rlx_alltoall(x, p, y2, p, m, n, F, FP8, stream)),
         ]
 
 
