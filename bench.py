@@ -423,6 +423,10 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
     }
     if world == 1 and not args.only and not args.no_latency:
         res["small_messages"] = small_message_latency(dev)
+    if world == 1 and not args.only and not args.no_workloads:
+        del ops, batch_ops, batches, step
+        torch.cuda.empty_cache()
+        res["workloads"] = workload_suite(dev, peak)
     if count != COUNT or args.only:
         res["config"]["workload"] = "PROFILING CASE, not the benchmark: %s on N=8 x fp32[%d]" % (
             ",".join(bytes_), count)
@@ -495,6 +499,123 @@ def small_message_latency(dev, reps: int = 200, graph_reps: int = 50) -> dict:
                 row["%s_%s" % (algo, wname)] = {"us_direct": round(direct, 2),
                                                 "us_graph": round(graphed, 2)}
         res[name] = row
+    return res
+
+
+# ------------------------------------------------- the other workloads
+
+def _timed_us(call, stream, reps: int, warmup: int = 3) -> float:
+    """Mean microseconds per call of `reps` back-to-back calls (CUDA events
+    at the two ends, on the launching stream)."""
+    import torch
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps * 1e3
+
+
+def _cold_us(call, stream, flush, reps: int) -> float:
+    """Median microseconds of one call with the L2 flushed before it (a
+    write of a buffer larger than L2 between calls, outside the events)."""
+    import torch
+    call()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1e3)
+    return statistics.median(ts)
+
+
+def workload_suite(dev, peak: float, reps: int = 20) -> dict:
+    """Per-operation figures on the other full-size workloads, drawn on the
+    device (same recipes as the host draws): decode bf16 [32, 8192] x 8 with
+    the L2 cold, prefill bf16 [4096, 8192] x 8 (DDA-tree and -flat, both
+    wires) and lp-collectives fp32 [67,108,864] x 8 (reduce-scatter,
+    all-gather, alltoall and quantise, both wires)."""
+    import torch
+    from precision_collective_reduction_fp32_b200 import binding as B
+    from precision_collective_reduction_fp32_b200 import synth
+    st = torch.cuda.current_stream(dev)
+    sp = st.cuda_stream or None
+    NAT, FP8, SUM = B.RLX_WIRE_NATIVE, B.RLX_WIRE_FP8_E4M3, B.RLX_SUM
+    wires = (("native", NAT), ("fp8", FP8))
+    res = {}
+
+    def entry(us, nbytes):
+        gbs = nbytes / (us * 1e-6) / 1e9
+        return {"us": round(us, 2), "GB/s": round(gbs, 1), "frac": round(gbs / peak, 3),
+                "MiB": round(nbytes / MIB, 2), "floor_us": round(nbytes / (peak * 1e9) * 1e6, 2)}
+
+    def allreduces(x, dcode, esize, cold=None):
+        n, c = x.shape
+        out = torch.empty_like(x)
+        ws = torch.empty(max(B.rlx_workspace_bytes(B.RLX_COLL_ALLREDUCE_TREE, c, n, dcode, FP8), 16),
+                         dtype=torch.uint8, device=dev)
+        ob = op_bytes(c, n, esize)
+        row = {}
+        for algo in ("flat", "tree"):
+            for wname, wire in wires:
+                if algo == "flat":
+                    f = lambda w=wire: B.rlx_allreduce_flat(x.data_ptr(), out.data_ptr(), c, c, n,
+                                                            dcode, w, SUM, sp)
+                else:
+                    f = lambda w=wire: B.rlx_allreduce_tree(x.data_ptr(), out.data_ptr(), c, c, n,
+                                                            dcode, w, SUM, ws.data_ptr(),
+                                                            ws.numel(), sp)
+                nb = ob["allreduce_%s_%s" % (algo, wname)]
+                us = _cold_us(f, st, cold, reps) if cold is not None else _timed_us(f, st, reps)
+                row["allreduce_%s_%s" % (algo, wname)] = entry(us, nb)
+        del out, ws
+        return row
+
+    # decode, L2 cold (the hot-L2 figures are under small_messages)
+    flush = torch.empty(256 * MIB, dtype=torch.uint8, device=dev)
+    x = synth.device_rank_buffers(2, dev)
+    res["decode_bf16_8x32x8192_cold_l2"] = allreduces(x, B.RLX_BF16, 2, cold=flush)
+    del x, flush
+    # prefill
+    x = synth.device_rank_buffers(3, dev)
+    res["prefill_bf16_8x4096x8192"] = allreduces(x, B.RLX_BF16, 2)
+    del x
+    # lp-collectives
+    x = synth.device_rank_buffers(5, dev)
+    n, c = x.shape
+    m = c // n
+    ob = op_bytes(c, n)
+    y = torch.empty_like(x)
+    rs = torch.empty((n, m), dtype=torch.float32, device=dev)
+    codes = torch.empty((n, c), dtype=torch.uint8, device=dev)
+    scales = torch.empty((n, (c + BLOCK - 1) // BLOCK), dtype=torch.float32, device=dev)
+    F = B.RLX_F32
+    row = {}
+    row["quantize_fp8"] = entry(_timed_us(lambda: B.rlx_quantize_fp8(
+        x.data_ptr(), F, n, c, c, codes.data_ptr(), scales.data_ptr(), sp), st, reps),
+        ob["quantize_fp8"])
+    for wname, wire in wires:
+        row["reduce_scatter_" + wname] = entry(_timed_us(lambda: B.rlx_reduce_scatter(
+            x.data_ptr(), c, rs.data_ptr(), m, m, n, F, wire, SUM, sp), st, reps),
+            ob["reduce_scatter_" + wname])
+        row["all_gather_" + wname] = entry(_timed_us(lambda: B.rlx_all_gather(
+            rs.data_ptr(), m, y.data_ptr(), c, m, n, F, wire, sp), st, reps),
+            ob["all_gather_" + wname])
+        row["alltoall_" + wname] = entry(_timed_us(lambda: B.rlx_alltoall(
+            x.data_ptr(), c, y.data_ptr(), c, m, n, F, wire, sp), st, reps),
+            ob["alltoall_" + wname])
+    res["lp_collectives_fp32_8x67108864"] = row
+    del x, y, rs, codes, scales
+    torch.cuda.empty_cache()
     return res
 
 
@@ -576,6 +697,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-latency", action="store_true",
                     help="skip the small-message latency figures")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the per-operation figures on the other workloads")
     ap.add_argument("--count", type=int, default=COUNT,
                     help="elements per rank (profiling cases only; the benchmark is 16,777,216)")
     ap.add_argument("--only", default="",

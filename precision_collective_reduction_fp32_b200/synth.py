@@ -61,26 +61,29 @@ def seed(workload: int, rank: int) -> int:
     return 1000 * workload + rank
 
 
-def draw_row(dist: str, count: int, s: int, std: float = 1.0) -> np.ndarray:
-    """One rank's fp32 values."""
-    g = torch.Generator().manual_seed(s)
+def _draw(dist: str, count: int, g: torch.Generator, std: float, device) -> torch.Tensor:
     if dist == "normal":
-        x = torch.randn(count, generator=g, dtype=torch.float32) * std
+        x = torch.randn(count, generator=g, dtype=torch.float32, device=device) * std
     elif dist == "normal_outliers":
-        x = torch.randn(count, generator=g, dtype=torch.float32) * std
-        hit = torch.rand(count, generator=g) < 0.01
+        x = torch.randn(count, generator=g, dtype=torch.float32, device=device) * std
+        hit = torch.rand(count, generator=g, device=device) < 0.01
         x = torch.where(hit, x * 100.0, x)
     elif dist == "student_t3":
-        x = torch.empty(count, dtype=torch.float32)
+        x = torch.empty(count, dtype=torch.float32, device=device)
         step = 1 << 24
         for lo in range(0, count, step):
             n = min(step, count - lo)
-            z = torch.randn(n, generator=g, dtype=torch.float64)
-            c = torch.randn((3, n), generator=g, dtype=torch.float64).square().sum(0)
+            z = torch.randn(n, generator=g, dtype=torch.float64, device=device)
+            c = torch.randn((3, n), generator=g, dtype=torch.float64, device=device).square().sum(0)
             x[lo:lo + n] = (z / torch.sqrt(c / 3.0)).to(torch.float32)
     else:
         raise ValueError(dist)
-    return x.numpy()
+    return x
+
+
+def draw_row(dist: str, count: int, s: int, std: float = 1.0) -> np.ndarray:
+    """One rank's fp32 values."""
+    return _draw(dist, count, torch.Generator().manual_seed(s), std, "cpu").numpy()
 
 
 def as_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -109,6 +112,21 @@ def rank_buffers(workload: int, count: int | None = None, nranks: int | None = N
     for r in range(nranks):
         x = draw_row(w.dist, count, seed(workload, r), w.std)
         out[r, :count] = x if dtype == "f32" else as_bf16_bits(x)
+    return out
+
+
+def device_rank_buffers(workload: int, device, salt: int = 0) -> torch.Tensor:
+    """[nranks, count] torch tensor of a workload drawn directly on a CUDA
+    device (fp32, or bf16 rounded from fp32), for timing at full size where
+    the host draw would take a minute.  Same recipe as rank_buffers, drawn
+    from the device's generator seeded with seed(workload, rank) + salt, so
+    the values follow the same distribution but are not the host bytes."""
+    w = WORKLOADS[workload]
+    out = torch.empty((w.nranks, w.count), dtype=torch.float32 if w.dtype == "f32"
+                      else torch.bfloat16, device=device)
+    for r in range(w.nranks):
+        g = torch.Generator(device=device).manual_seed(seed(workload, r) + salt)
+        out[r].copy_(_draw(w.dist, w.count, g, w.std, device))
     return out
 
 
