@@ -118,6 +118,69 @@ __device__ __forceinline__ void store4(T *p, int valid, const float (&v)[4]) {
     }
 }
 
+// Four consecutive elements kept as loaded (fp32: 4 words, bf16: 2 words),
+// widened to fp32 only where they are used; invalid elements hold +0.
+template <typename T> struct Raw4;
+template <> struct Raw4<float> { uint4 w; };
+template <> struct Raw4<uint16_t> { uint2 w; };
+
+template <typename T, bool VEC>
+__device__ __forceinline__ Raw4<T> load_raw4(const T *p, int valid) {
+    Raw4<T> r;
+    if constexpr (sizeof(T) == 4) {
+        if (VEC && valid == 4) {
+            r.w = ld_stream(reinterpret_cast<const uint4 *>(p));
+        } else {
+            uint32_t w[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) w[k] = k < valid ? __float_as_uint(Elem<T>::load(p + k)) : 0u;
+            r.w = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    } else {
+        if (VEC && valid == 4) {
+            r.w = ld_stream(reinterpret_cast<const uint2 *>(p));
+        } else {
+            uint32_t w[2] = {0u, 0u};
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                if (k < valid)
+                    w[k / 2] |= static_cast<uint32_t>(ld_stream(reinterpret_cast<const unsigned short *>(p) + k))
+                                << (16 * (k % 2));
+            r.w = make_uint2(w[0], w[1]);
+        }
+    }
+    return r;
+}
+
+template <typename T> __device__ __forceinline__ Raw4<T> raw4_zero() {
+    Raw4<T> r;
+    if constexpr (sizeof(T) == 4) r.w = make_uint4(0u, 0u, 0u, 0u);
+    else r.w = make_uint2(0u, 0u);
+    return r;
+}
+
+__device__ __forceinline__ void widen4(const Raw4<float> &r, float (&v)[4]) {
+    v[0] = __uint_as_float(r.w.x); v[1] = __uint_as_float(r.w.y);
+    v[2] = __uint_as_float(r.w.z); v[3] = __uint_as_float(r.w.w);
+}
+__device__ __forceinline__ void widen4(const Raw4<uint16_t> &r, float (&v)[4]) {
+    v[0] = __uint_as_float(r.w.x << 16); v[1] = __uint_as_float(r.w.x & 0xffff0000u);
+    v[2] = __uint_as_float(r.w.y << 16); v[3] = __uint_as_float(r.w.y & 0xffff0000u);
+}
+
+// Bits of max |v| over the four elements (a non-negative float's bits; for
+// those the integer order is the value order).  bf16 magnitudes are compared
+// as 16-bit integers two at a time.
+__device__ __forceinline__ uint32_t absmax4_bits(const Raw4<float> &r) {
+    const float m = fmaxf(fmaxf(fabsf(__uint_as_float(r.w.x)), fabsf(__uint_as_float(r.w.y))),
+                          fmaxf(fabsf(__uint_as_float(r.w.z)), fabsf(__uint_as_float(r.w.w))));
+    return __float_as_uint(m);
+}
+__device__ __forceinline__ uint32_t absmax4_bits(const Raw4<uint16_t> &r) {
+    const uint32_t m = __vmaxu2(r.w.x & 0x7fff7fffu, r.w.y & 0x7fff7fffu);
+    return max(m & 0xffffu, m >> 16) << 16;
+}
+
 // --------------------------------------------------------------- E4M3 codec
 
 // Two fp32 -> two E4M3 codes (round to nearest even, saturating to +-448,
@@ -207,8 +270,9 @@ __device__ __forceinline__ float quotient_rn(float x, float s, float y) {
 
 // Blackwell executes two fp32 lanes per instruction (add/mul/fma .f32x2);
 // each lane rounds exactly like the scalar instruction, so the packed forms
-// below give the same bits with half the instructions.  RLX_PACKED_F32X2=0
-// selects the scalar forms.
+// below give the same bits with half the instructions.  A packed product is
+// never the addend of a packed add here (such a pair gets fused, see
+// dequant4).  RLX_PACKED_F32X2=0 selects the scalar forms.
 #ifndef RLX_PACKED_F32X2
 #define RLX_PACKED_F32X2 1
 #endif
@@ -226,14 +290,6 @@ __device__ __forceinline__ float2 quotient_rn2(float2 x, float s, float y) {
     return __ffma2_rn(r, ny2, q);
 #else
     return f2(quotient_rn(x.x, s, y), quotient_rn(x.y, s, y));
-#endif
-}
-
-__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
-#if RLX_PACKED_F32X2
-    return __fmul2_rn(a, b);
-#else
-    return f2(__fmul_rn(a.x, b.x), __fmul_rn(a.y, b.y));
 #endif
 }
 
@@ -263,11 +319,24 @@ __device__ __forceinline__ uint32_t quant4(const float (&v)[4], Scale sc) {
     return e4m3x4_from_f32(q);
 }
 
-// Dequantise 4 packed codes with scale s: fl32(e4m3(code) * s).
+// quant4 for a block whose scale takes the fast quotient (sc.y != 0).
+__device__ __forceinline__ uint32_t quant4_fast(const float (&v)[4], Scale sc) {
+    const float2 a = quotient_rn2(f2(v[0], v[1]), sc.s, sc.y);
+    const float2 b = quotient_rn2(f2(v[2], v[3]), sc.s, sc.y);
+    const float q[4] = {a.x, a.y, b.x, b.y};
+    return e4m3x4_from_f32(q);
+}
+
+// Dequantise 4 packed codes with scale s: fl32(e4m3(code) * s).  The
+// multiply is the scalar __fmul_rn, which is never merged into an FMA: a
+// packed multiply whose product fed a packed add was contracted into a packed
+// FMA by this toolchain (even as PTX mul.rn.f32x2 / add.rn.f32x2), which skips
+// the rounding of the product that the definition requires.
 __device__ __forceinline__ void dequant4(uint32_t codes, float s, float (&y)[4]) {
-    const float2 a = mul2_rn(e4m3x2_to_f32(codes & 0xffffu), f2(s, s));
-    const float2 b = mul2_rn(e4m3x2_to_f32(codes >> 16), f2(s, s));
-    y[0] = a.x; y[1] = a.y; y[2] = b.x; y[3] = b.y;
+    const float2 a = e4m3x2_to_f32(codes & 0xffffu);
+    const float2 b = e4m3x2_to_f32(codes >> 16);
+    y[0] = __fmul_rn(a.x, s); y[1] = __fmul_rn(a.y, s);
+    y[2] = __fmul_rn(b.x, s); y[3] = __fmul_rn(b.y, s);
 }
 
 // What a receiver holds after K 128-blocks crossed the FP8 wire.  The warp
@@ -353,6 +422,14 @@ __device__ __forceinline__ void for_each_unit(uint32_t total, F &&f) {
 template <typename F>
 __device__ __forceinline__ void with_full(bool full, F &&f) {
     if (full) f(std::true_type{});
+    else f(std::false_type{});
+}
+
+// Calls f(std::true_type{}) when every block scale of the unit takes the fast
+// quotient, else f(std::false_type{}).
+template <typename F>
+__device__ __forceinline__ void with_fast(bool fast, F &&f) {
+    if (fast) f(std::true_type{});
     else f(std::false_type{});
 }
 

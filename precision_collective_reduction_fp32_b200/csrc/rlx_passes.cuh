@@ -110,31 +110,127 @@ __device__ __forceinline__ void reduce_vec(const T *src, size_t pitch, int n, in
 
 // ---------------------------------------------------- FP8 wire, warp per block
 
-// acc = SUM_s wire(x_s) over the 128-block at `src` in each of n rows, 4
-// elements per lane (`valid` of them real; the rest +0).
-template <typename T, int NR, bool VEC>
-__device__ __forceinline__ void reduce_block_fp8(const T *src, size_t pitch, int n, int valid,
-                                                 float (&acc)[4]) {
-    float x[NR][4];
+// 128-blocks a warp reduces at once on the FP8 wire: a bf16 block is half the
+// bytes of an fp32 one, so a bf16 unit takes two adjacent blocks and a warp
+// has as many bytes in flight per unit for either type.
+#ifndef RLX_BPU_BF16
+#define RLX_BPU_BF16 2
+#endif
+template <typename T> constexpr int kBpu = sizeof(T) == 2 ? RLX_BPU_BF16 : 1;
+// 1: one warp vote per unit selects branch-free quantisation when every
+// block scale takes the fast quotient; 0: every block branches on its scale.
+#ifndef RLX_FAST_VOTE
+#define RLX_FAST_VOTE 1
+#endif
+
+// acc[j] = SUM_s wire(x_s) over the BPU adjacent 128-blocks at src + 128 j in
+// each of n rows, 4 elements per lane (valid[j] of them real; the rest +0).
+// Every (rank, block) pair is one FP8 block: its amax is one warp
+// reduction, and lane l computes the scale of pair l % (NR*BPU), which is
+// broadcast just before that pair is quantised.  The loads stay raw until
+// then, so a bf16 pair costs 2 registers.
+template <typename T, int NR, bool VEC, int BPU>
+__device__ __forceinline__ void reduce_blocks_fp8(const T *src, size_t pitch, int n,
+                                                  const int (&valid)[BPU],
+                                                  float (&acc)[BPU][4]) {
+    constexpr int K = NR * BPU;
+    static_assert(K <= 32 && (K & (K - 1)) == 0, "NR * BPU must be a power of two <= 32");
     const int e0 = lane_id() * 4;
+    Raw4<T> x[NR][BPU];
 #pragma unroll
-    for (int s = 0; s < NR; ++s) {
-        if (s < n) {
-            load4<T, VEC>(src + s * pitch + e0, valid, x[s]);
-        } else {
+    for (int s = 0; s < NR; ++s)
 #pragma unroll
-            for (int k = 0; k < 4; ++k) x[s][k] = 0.0f;
+        for (int j = 0; j < BPU; ++j)
+            x[s][j] = s < n ? load_raw4<T, VEC>(src + s * pitch + j * kBlock + e0, valid[j])
+                            : raw4_zero<T>();
+    const int mine = threadIdx.x & (K - 1);
+    uint32_t a = 0u;
+#pragma unroll
+    for (int s = 0; s < NR; ++s)
+#pragma unroll
+        for (int j = 0; j < BPU; ++j) {
+            const uint32_t m = __reduce_max_sync(kFull, absmax4_bits(x[s][j]));
+            if (mine == s * BPU + j) a = m;
+        }
+    const Scale own = make_scale(__uint_as_float(a));
+    // one vote: when every scale of the unit takes the fast quotient (the
+    // usual case) the quantisation below is straight-line code the compiler
+    // can interleave across blocks
+    with_fast(RLX_FAST_VOTE && __all_sync(kFull, own.y != 0.0f), [&](auto fast) {
+#pragma unroll
+        for (int s = 0; s < NR; ++s) {
+            if (s < n) {
+#pragma unroll
+                for (int j = 0; j < BPU; ++j) {
+                    Scale sc;
+                    sc.s = __shfl_sync(kFull, own.s, s * BPU + j);
+                    sc.y = __shfl_sync(kFull, own.y, s * BPU + j);
+                    float v[4];
+                    widen4(x[s][j], v);
+                    dequant4(decltype(fast)::value ? quant4_fast(v, sc) : quant4(v, sc), sc.s, v);
+                    if (s == 0) {
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) acc[j][k] = v[k];
+                    } else {
+                        const float2 lo = add2_rn(f2(acc[j][0], acc[j][1]), f2(v[0], v[1]));
+                        const float2 hi = add2_rn(f2(acc[j][2], acc[j][3]), f2(v[2], v[3]));
+                        acc[j][0] = lo.x; acc[j][1] = lo.y; acc[j][2] = hi.x; acc[j][3] = hi.y;
+                    }
+                }
+            }
+        }
+    });
+}
+
+// ------------------------------------------------------ 16-byte bf16 stores
+
+// Two fp32 values -> two bf16 (round to nearest even) in one word, `lo` in the
+// low half.
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// Row pieces of 16 bytes for a bf16 block pair held as 4 values per lane per
+// block: lane 2i gets elements [8i, 8i+8) of block 0 and lane 2i+1 the same
+// elements of block 1 (one exchange with the neighbouring lane), so a warp
+// writes the pair with one 16-byte store per lane instead of two of 8 bytes.
+// The piece of lane l starts at element bf16_piece(l) of the pair.
+__device__ __forceinline__ uint4 bf16_pair_pieces(const float (&v)[2][4]) {
+    const uint2 w0 = make_uint2(bf16x2_bits(v[0][0], v[0][1]), bf16x2_bits(v[0][2], v[0][3]));
+    const uint2 w1 = make_uint2(bf16x2_bits(v[1][0], v[1][1]), bf16x2_bits(v[1][2], v[1][3]));
+    const bool odd = lane_id() & 1;
+    const uint2 give = odd ? w0 : w1;
+    const uint2 got = make_uint2(__shfl_xor_sync(kFull, give.x, 1), __shfl_xor_sync(kFull, give.y, 1));
+    return odd ? make_uint4(got.x, got.y, w1.x, w1.y) : make_uint4(w0.x, w0.y, got.x, got.y);
+}
+__device__ __forceinline__ int bf16_piece(int lane) { return (lane & 1) * kBlock + (lane >> 1) * 8; }
+
+// May the rows at p (pitch `pitch` elements of T) take 16-byte bf16 stores
+// at block-pair offsets?
+template <typename T>
+__device__ __forceinline__ bool rows_16b(const T *p, size_t pitch) {
+    return sizeof(T) == 2 && ((reinterpret_cast<uintptr_t>(p) | pitch * sizeof(T)) & 15) == 0;
+}
+
+// Stores the reduced blocks of a unit (acc[j] = block j, 4 values per lane) at
+// dst + 128 j in each of `rows` rows `pitch` apart.  A full bf16 block pair
+// on 16-byte aligned rows goes out as 16-byte pieces.
+template <typename T, bool VEC, int BPU, typename Full>
+__device__ __forceinline__ void store_blocks(T *dst, size_t pitch, int rows, Full, bool wide,
+                                             const int (&valid)[BPU], const float (&acc)[BPU][4]) {
+    if constexpr (BPU == 2 && sizeof(T) == 2 && Full::value) {
+        if (VEC && wide) {
+            const uint4 q = bf16_pair_pieces(acc);
+            T *p = dst + bf16_piece(lane_id());
+            for (int r = 0; r < rows; ++r) st_stream(reinterpret_cast<uint4 *>(p + r * pitch), q);
+            return;
         }
     }
-    wire_fp8_blocks<NR>(x);
-    float2 a01 = f2(x[0][0], x[0][1]), a23 = f2(x[0][2], x[0][3]);
+    const int e0 = lane_id() * 4;
+    for (int r = 0; r < rows; ++r)
 #pragma unroll
-    for (int s = 1; s < NR; ++s)
-        if (s < n) {
-            a01 = add2_rn(a01, f2(x[s][0], x[s][1]));
-            a23 = add2_rn(a23, f2(x[s][2], x[s][3]));
-        }
-    acc[0] = a01.x; acc[1] = a01.y; acc[2] = a23.x; acc[3] = a23.y;
+        for (int j = 0; j < BPU; ++j) store4<T, VEC>(dst + r * pitch + j * kBlock + e0, valid[j], acc[j]);
 }
 
 // Valid elements of a vector starting at element i0 of a segment ending at
@@ -281,23 +377,39 @@ __device__ __forceinline__ void tree_reduce_native_unit(uint32_t g, const T *sen
     });
 }
 
-// Pass 1, FP8: unit b = 128-block b; reduce, then quantise the reduced block
-// again into the payload (codes padded to whole blocks, one scale per block).
+// Pass 1, FP8: unit u = the BPU blocks from block u*BPU on; reduce, then
+// quantise each reduced block again into the payload (codes padded to whole
+// blocks, one scale per block).
 template <typename T, int NR, bool VEC>
-__device__ __forceinline__ void tree_reduce_fp8_unit(uint32_t b, const T *send, size_t count,
+__device__ __forceinline__ void tree_reduce_fp8_unit(uint32_t u, const T *send, size_t count,
                                                      size_t stride, int n, uint8_t *ws_codes,
                                                      float *ws_scales) {
+    constexpr int BPU = kBpu<T>;
     const int e0 = lane_id() * 4;
-    const size_t base = static_cast<size_t>(b) * kBlock;
-    with_full(base + kBlock <= count, [&](auto full) {
-        const int valid = decltype(full)::value ? 4 : lane_valid(base, count);
-        float acc[4];
-        reduce_block_fp8<T, NR, VEC>(send + base, stride, n, valid, acc);
-        const Scale sc = make_scale(warp_amax4(acc));
-        const uint32_t codes = quant4(acc, sc);
-        // default caching: pass 2 reads the payload back right away
-        *reinterpret_cast<uint32_t *>(ws_codes + base + e0) = codes;
-        if (lane_id() == 0) ws_scales[b] = sc.s;
+    const size_t base = static_cast<size_t>(u) * BPU * kBlock;
+    with_full(base + BPU * kBlock <= count, [&](auto full) {
+        int valid[BPU];
+#pragma unroll
+        for (int j = 0; j < BPU; ++j)
+            valid[j] = decltype(full)::value ? 4 : lane_valid(base + j * kBlock, count);
+        float acc[BPU][4];
+        reduce_blocks_fp8<T, NR, VEC, BPU>(send + base, stride, n, valid, acc);
+        float amax[BPU];
+#pragma unroll
+        for (int j = 0; j < BPU; ++j) amax[j] = warp_amax4(acc[j]);
+        Scale sc[BPU];
+        if constexpr (BPU == 1) sc[0] = make_scale(amax[0]);
+        else make_scales<BPU>(amax, sc);
+#pragma unroll
+        for (int j = 0; j < BPU; ++j) {
+            const size_t bj = base + j * kBlock;
+            if (decltype(full)::value || bj < count) {
+                const uint32_t codes = quant4(acc[j], sc[j]);
+                // default caching: pass 2 reads the payload back right away
+                *reinterpret_cast<uint32_t *>(ws_codes + bj + e0) = codes;
+                if (lane_id() == 0) ws_scales[bj / kBlock] = sc[j].s;
+            }
+        }
     });
 }
 
@@ -332,6 +444,33 @@ __device__ __forceinline__ void tree_gather_fp8_unit(uint32_t g, T *recv, size_t
     const size_t nblk = (count + kBlock - 1) / kBlock;
     const int e0 = lane_id() * 4;
     const size_t b0 = static_cast<size_t>(g) * kJd;
+    if constexpr (sizeof(T) == 2 && VEC && kJd % 2 == 0) {
+        // bf16 on 16-byte aligned rows, whole unit: lane l takes elements
+        // [8l, 8l+8) of every block pair (half-warp l / 16 per block), so each
+        // row gets one 16-byte store per lane per pair
+        if ((b0 + kJd) * kBlock <= count && rows_16b(recv, stride)) {
+            const int l = lane_id();
+            uint4 q[kJd / 2];
+#pragma unroll
+            for (int p = 0; p < kJd / 2; ++p) {
+                const size_t b = b0 + 2 * p + (l >> 4);
+                const uint2 codes = __ldcg(reinterpret_cast<const uint2 *>(ws_codes + (b0 + 2 * p) * kBlock + 8 * l));
+                const float s = __ldcg(ws_scales + b);
+                float y[2][4];
+                dequant4(codes.x, s, y[0]);
+                dequant4(codes.y, s, y[1]);
+                q[p] = make_uint4(bf16x2_bits(y[0][0], y[0][1]), bf16x2_bits(y[0][2], y[0][3]),
+                                  bf16x2_bits(y[1][0], y[1][1]), bf16x2_bits(y[1][2], y[1][3]));
+            }
+            for (int r = 0; r < n; ++r) {
+                T *dst = recv + r * stride + b0 * kBlock + 8 * l;
+#pragma unroll
+                for (int p = 0; p < kJd / 2; ++p)
+                    st_stream(reinterpret_cast<uint4 *>(dst + 2 * p * kBlock), q[p]);
+            }
+            return;
+        }
+    }
     with_full((b0 + kJd) * kBlock <= count, [&](auto full) {
         constexpr bool F = decltype(full)::value;
         const uint8_t *cp = ws_codes + b0 * kBlock + e0;

@@ -14,9 +14,10 @@
 //   native wire: one thread per 16-byte vector of each row (4 fp32 or 8 bf16);
 //     the thread loads that vector from all N ranks before adding, so N
 //     16-byte loads are in flight per thread;
-//   FP8 wire: one warp per 128-element block, 4 elements per lane, so a block
-//     amax is one warp reduction; the warp loads the block from all N ranks,
-//     dequantises each rank's quantised block and sums in rank order.
+//   FP8 wire: one warp per 128-element block (two adjacent blocks for bf16),
+//     4 elements per lane per block, so a block amax is one warp reduction;
+//     the warp loads its blocks from all N ranks, dequantises each rank's
+//     quantised block and sums in rank order.
 // Units of work are numbered in memory order (chunk-major for chunked
 // passes) and handed out in CTA-sized runs by for_each_unit, so the CTAs in
 // flight stream one compact stretch of every row.
@@ -56,11 +57,15 @@ constexpr int kPfFlat = RLX_P_FP8_FLAT;
 #ifndef RLX_MINB_FP8
 #define RLX_MINB_FP8 4
 #endif
+#ifndef RLX_MINB_FP8_BF16
+#define RLX_MINB_FP8_BF16 4
+#endif
 #ifndef RLX_MINB_FP8_FLAT
-#define RLX_MINB_FP8_FLAT 3
+#define RLX_MINB_FP8_FLAT 4
 #endif
 template <int NR> constexpr int kMinBlocksNative = NR <= 8 ? RLX_MINB_NATIVE : 1;
-template <int NR> constexpr int kMinBlocksFp8 = NR <= 8 ? RLX_MINB_FP8 : 1;
+template <typename T, int NR>
+constexpr int kMinBlocksFp8 = NR > 8 ? 1 : sizeof(T) == 2 ? RLX_MINB_FP8_BF16 : RLX_MINB_FP8;
 template <int NR> constexpr int kMinBlocksFp8Flat = NR <= 8 ? RLX_MINB_FP8_FLAT : 1;
 
 // DDA-flat, native: unit g = 32 consecutive 16-byte vectors (lane l: 32g + l).
@@ -82,19 +87,23 @@ flat_native_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
     });
 }
 
-// DDA-flat, FP8: unit g = 128-block g.
+// DDA-flat, FP8: unit u = the kBpu<T> blocks from block u*kBpu<T> on.
 template <typename T, int NR, bool VEC>
 __global__ void __launch_bounds__(kThreads, kMinBlocksFp8Flat<NR>)
 flat_fp8_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
-    const uint32_t nblk = static_cast<uint32_t>((count + kBlock - 1) / kBlock);
-    const int e0 = lane_id() * 4;
-    for_each_unit<kPfFlat>(nblk, [&](uint32_t b) {
-        const size_t base = static_cast<size_t>(b) * kBlock;
-        with_full(base + kBlock <= count, [&](auto full) {
-            const int valid = decltype(full)::value ? 4 : lane_valid(base, count);
-            float acc[4];
-            reduce_block_fp8<T, NR, VEC>(send + base, stride, n, valid, acc);
-            for (int r = 0; r < n; ++r) store4<T, VEC>(recv + r * stride + base + e0, valid, acc);
+    constexpr int BPU = kBpu<T>;
+    const uint32_t units = static_cast<uint32_t>((count + BPU * kBlock - 1) / (BPU * kBlock));
+    const bool wide = rows_16b(recv, stride);
+    for_each_unit<kPfFlat>(units, [&](uint32_t u) {
+        const size_t base = static_cast<size_t>(u) * BPU * kBlock;
+        with_full(base + BPU * kBlock <= count, [&](auto full) {
+            int valid[BPU];
+#pragma unroll
+            for (int j = 0; j < BPU; ++j)
+                valid[j] = decltype(full)::value ? 4 : lane_valid(base + j * kBlock, count);
+            float acc[BPU][4];
+            reduce_blocks_fp8<T, NR, VEC, BPU>(send + base, stride, n, valid, acc);
+            store_blocks<T, VEC, BPU>(recv + base, stride, n, full, wide, valid, acc);
         });
     });
 }
@@ -112,12 +121,13 @@ tree_reduce_native_kernel(const T *send, T *recv, size_t count, size_t stride, i
 
 // DDA-tree pass 1, FP8.
 template <typename T, int NR, bool VEC, int P>
-__global__ void __launch_bounds__(kThreads, kMinBlocksFp8<NR>)
+__global__ void __launch_bounds__(kThreads, kMinBlocksFp8<T, NR>)
 tree_reduce_fp8_kernel(const T *send, size_t count, size_t stride, int n,
                        uint8_t *ws_codes, float *ws_scales) {
-    const uint32_t nblk = static_cast<uint32_t>((count + kBlock - 1) / kBlock);
-    for_each_unit<P>(nblk, [&](uint32_t b) {
-        tree_reduce_fp8_unit<T, NR, VEC>(b, send, count, stride, n, ws_codes, ws_scales);
+    constexpr int BPU = kBpu<T>;
+    const uint32_t units = static_cast<uint32_t>((count + BPU * kBlock - 1) / (BPU * kBlock));
+    for_each_unit<P>(units, [&](uint32_t u) {
+        tree_reduce_fp8_unit<T, NR, VEC>(u, send, count, stride, n, ws_codes, ws_scales);
     });
 }
 
@@ -142,22 +152,26 @@ rs_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t 
     });
 }
 
-// ReduceScatter, FP8: unit = (destination rank r, 128-block of chunk r);
-// blocks anchored at the chunk start r*m.
+// ReduceScatter, FP8: unit = (destination rank r, kBpu<T> adjacent blocks of
+// chunk r); blocks anchored at the chunk start r*m.
 template <typename T, int NR, bool VEC, int P>
-__global__ void __launch_bounds__(kThreads, kMinBlocksFp8<NR>)
+__global__ void __launch_bounds__(kThreads, kMinBlocksFp8<T, NR>)
 rs_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n,
               FastDiv per_chunk) {
+    constexpr int BPU = kBpu<T>;
     const uint32_t units = per_chunk.d * static_cast<uint32_t>(n);
-    const int e0 = lane_id() * 4;
+    const bool wide = rows_16b(recv, rstride);
     for_each_unit<P>(units, [&](uint32_t g) {
         const uint32_t r = fast_div(g, per_chunk);
-        const size_t j0 = static_cast<size_t>(g - r * per_chunk.d) * kBlock;
-        with_full(j0 + kBlock <= m, [&](auto full) {
-            const int valid = decltype(full)::value ? 4 : lane_valid(j0, m);
-            float acc[4];
-            reduce_block_fp8<T, NR, VEC>(send + r * m + j0, sstride, n, valid, acc);
-            store4<T, VEC>(recv + r * rstride + j0 + e0, valid, acc);
+        const size_t j0 = static_cast<size_t>(g - r * per_chunk.d) * BPU * kBlock;
+        with_full(j0 + BPU * kBlock <= m, [&](auto full) {
+            int valid[BPU];
+#pragma unroll
+            for (int j = 0; j < BPU; ++j)
+                valid[j] = decltype(full)::value ? 4 : lane_valid(j0 + j * kBlock, m);
+            float acc[BPU][4];
+            reduce_blocks_fp8<T, NR, VEC, BPU>(send + r * m + j0, sstride, n, valid, acc);
+            store_blocks<T, VEC, BPU>(recv + r * rstride + j0, rstride, 1, full, wide, valid, acc);
         });
     });
 }
@@ -202,8 +216,8 @@ cudaError_t launch_allreduce_flat(const void *send, void *recv, size_t count, si
             return launch(flat_native_kernel<T, NR, VEC>, units, kWarps * kPn, stream, s, r,
                           count, stride, nranks);
         }
-        const size_t nblk = (count + kBlock - 1) / kBlock;
-        return launch(flat_fp8_kernel<T, NR, VEC>, nblk, kWarps * kPfFlat, stream, s, r, count,
+        const size_t units = (count + kBpu<T> * kBlock - 1) / (kBpu<T> * kBlock);
+        return launch(flat_fp8_kernel<T, NR, VEC>, units, kWarps * kPfFlat, stream, s, r, count,
                       stride, nranks);
     });
 }
@@ -223,10 +237,11 @@ cudaError_t launch_tree_reduce(const void *send, void *recv, size_t count, size_
                           make_fastdiv(static_cast<uint32_t>(per)));
         }
         const size_t nblk = (count + kBlock - 1) / kBlock;
+        const size_t units = (nblk + kBpu<T> - 1) / kBpu<T>;
         if (nblk < RLX_FP8_SMALL_BLOCKS)
-            return launch(tree_reduce_fp8_kernel<T, NR, VEC, 1>, nblk, kWarps, stream, s, count,
+            return launch(tree_reduce_fp8_kernel<T, NR, VEC, 1>, units, kWarps, stream, s, count,
                           stride, nranks, ws_codes, ws_scales);
-        return launch(tree_reduce_fp8_kernel<T, NR, VEC, kPf>, nblk, kWarps * kPf, stream, s,
+        return launch(tree_reduce_fp8_kernel<T, NR, VEC, kPf>, units, kWarps * kPf, stream, s,
                       count, stride, nranks, ws_codes, ws_scales);
     });
 }
@@ -238,14 +253,15 @@ cudaError_t launch_reduce_scatter(const void *send, size_t send_stride, void *re
         const T *s = static_cast<const T *>(send);
         T *r = static_cast<T *>(recv);
         const size_t nn = static_cast<size_t>(nranks);
-        const size_t per = wire == RLX_WIRE_NATIVE ? ((m + VecN<T>::n - 1) / VecN<T>::n + 31) / 32
-                                                   : (m + kBlock - 1) / kBlock;
+        const size_t per = wire == RLX_WIRE_NATIVE
+                               ? ((m + VecN<T>::n - 1) / VecN<T>::n + 31) / 32
+                               : (m + kBpu<T> * kBlock - 1) / (kBpu<T> * kBlock);
         if (per >= (size_t{1} << 32)) return cudaErrorInvalidValue;
         const FastDiv fd = make_fastdiv(static_cast<uint32_t>(per));
         if (wire == RLX_WIRE_NATIVE)
             return launch(rs_native_kernel<T, NR, VEC>, per * nn, kWarps * kPn, stream, s,
                           send_stride, r, recv_stride, m, nranks, fd);
-        if (per * nn < RLX_FP8_SMALL_BLOCKS)
+        if (per * kBpu<T> * nn < RLX_FP8_SMALL_BLOCKS)
             return launch(rs_fp8_kernel<T, NR, VEC, 1>, per * nn, kWarps, stream, s, send_stride,
                           r, recv_stride, m, nranks, fd);
         return launch(rs_fp8_kernel<T, NR, VEC, kPf>, per * nn, kWarps * kPf, stream, s,

@@ -134,6 +134,10 @@ def test_workload3_prefill_tree():
         t8 = _allreduce("tree", dx, count, wire, B.RLX_BF16)
         _check_allreduce_sampled(x, t8, "tree", wire, count, edges)
         assert _rows_identical(t8)
+        del t8
+        f8 = _allreduce("flat", dx, count, wire, B.RLX_BF16)
+        _check_allreduce_sampled(x, f8, "flat", wire, count, edges)
+        assert _rows_identical(f8)
 
 
 # ---------------------------------------------------------------- workload 4

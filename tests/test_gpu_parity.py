@@ -215,6 +215,27 @@ def test_tree_in_place_mid_size(wire, count, inplace):
 
 
 @pytest.mark.parametrize("algo", ["flat", "tree"])
+def test_bf16_fp8_large_ragged(algo):
+    """bf16 on the FP8 wire past the small-message threshold (>= 32768 blocks,
+    the multi-unit-per-warp launch) with an odd block count and a partial last
+    block, so the last two-block unit holds one partial block."""
+    count = 4_194_304 + 2 * 128 + 77
+    x = synth.rank_buffers(4, count=count, nranks=8, dtype="bf16")
+    got = _run_allreduce(algo, x, count, count, B.RLX_WIRE_FP8_E4M3)
+    fn = oracle.allreduce_flat if algo == "flat" else oracle.allreduce_tree
+    assert _bits_equal(got, fn(x, wire=oracle.FP8))
+
+
+def test_bf16_fp8_reduce_scatter_large_ragged():
+    """Reduce-scatter, bf16 on the FP8 wire: chunks of an odd number of
+    blocks with a partial last block, past the small-message threshold."""
+    n, m = 8, 524_288 + 128 + 5
+    x = synth.rank_buffers(5, count=n * m, nranks=n, dtype="bf16")
+    got = _chunked("rlx_reduce_scatter", x, m, n * m, m, m, B.RLX_WIRE_FP8_E4M3)
+    assert _bits_equal(got, oracle.reduce_scatter(x, m, wire=oracle.FP8, recv_stride=m))
+
+
+@pytest.mark.parametrize("algo", ["flat", "tree"])
 @pytest.mark.parametrize("wire", WIRES)
 @pytest.mark.parametrize("dtype", DTYPES)
 def test_one_rank_copies(algo, wire, dtype):
@@ -232,6 +253,28 @@ def test_worked_example(algo, wire, dtype):
         got = refpipe.bf16_to_f32(_run_allreduce(algo, x, 200, 200, wire)) if dtype == "bf16" \
             else _run_allreduce(algo, x, 200, 200, wire)
         assert np.all(got == nranks * (nranks - 1) / 2)
+
+
+@pytest.mark.parametrize("algo", ["flat", "tree"])
+@pytest.mark.parametrize("dtype", DTYPES)
+def test_allreduce_fp8_special_scales(algo, dtype):
+    """FP8 wire with ranks whose blocks take every scale path: all zeros
+    (scale 0), ordinary values, values so small that the scale is below the
+    fast-quotient bound (IEEE division), subnormal inputs, and huge values;
+    units mix fast and slow blocks, and later columns make some units all fast."""
+    n, count = 6, 5 * 256 + 77
+    x = synth.rank_buffers(4, count=count, nranks=n).astype(np.float64)
+    x[0] = 0.0
+    x[2] *= 1e-30
+    x[3] *= 1e-39
+    x[4] *= 1e30
+    x[5, :600] *= 1e-33
+    x = x.astype(np.float32)
+    if dtype == "bf16":
+        x = synth.as_bf16_bits(x)
+    got = _run_allreduce(algo, x, count, count, B.RLX_WIRE_FP8_E4M3)
+    fn = oracle.allreduce_flat if algo == "flat" else oracle.allreduce_tree
+    assert _bits_equal(got, fn(x, wire=oracle.FP8))
 
 
 def test_signed_zero():
