@@ -538,7 +538,7 @@ def _cold_us(call, stream, flush, reps: int) -> float:
     return statistics.median(ts)
 
 
-def workload_suite(dev, peak: float, reps: int = 20) -> dict:
+def workload_suite(dev, peak: float, reps: int = 20, scale: int = 1) -> dict:
     """Per-operation figures on the other full-size workloads, drawn on the
     device (same recipes as the host draws): decode bf16 [32, 8192] x 8 with
     the L2 cold, prefill bf16 [4096, 8192] x 8 (DDA-tree and -flat, both
@@ -552,6 +552,8 @@ def workload_suite(dev, peak: float, reps: int = 20) -> dict:
     NAT, FP8, SUM = B.RLX_WIRE_NATIVE, B.RLX_WIRE_FP8_E4M3, B.RLX_SUM
     wires = (("native", NAT), ("fp8", FP8))
     res = {}
+    # scale > 1 divides every workload's count (profiling cases only)
+    draw = lambda k: synth.device_rank_buffers(k, dev, count=synth.WORKLOADS[k].count // scale)
 
     def entry(us, nbytes):
         gbs = nbytes / (us * 1e-6) / 1e9
@@ -582,15 +584,15 @@ def workload_suite(dev, peak: float, reps: int = 20) -> dict:
 
     # decode, L2 cold (the hot-L2 figures are under small_messages)
     flush = torch.empty(256 * MIB, dtype=torch.uint8, device=dev)
-    x = synth.device_rank_buffers(2, dev)
+    x = draw(2)
     res["decode_bf16_8x32x8192_cold_l2"] = allreduces(x, B.RLX_BF16, 2, cold=flush)
     del x, flush
     # prefill
-    x = synth.device_rank_buffers(3, dev)
+    x = draw(3)
     res["prefill_bf16_8x4096x8192"] = allreduces(x, B.RLX_BF16, 2)
     del x
     # lp-collectives
-    x = synth.device_rank_buffers(5, dev)
+    x = draw(5)
     n, c = x.shape
     m = c // n
     ob = op_bytes(c, n)
@@ -699,6 +701,11 @@ def main(argv=None):
                     help="skip the small-message latency figures")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the per-operation figures on the other workloads")
+    ap.add_argument("--suite-only", action="store_true",
+                    help="profiling: run only the other workloads' per-operation figures "
+                         "(--steps calls each)")
+    ap.add_argument("--suite-scale", type=int, default=1,
+                    help="profiling: divide the other workloads' counts by this")
     ap.add_argument("--count", type=int, default=COUNT,
                     help="elements per rank (profiling cases only; the benchmark is 16,777,216)")
     ap.add_argument("--only", default="",
@@ -707,6 +714,15 @@ def main(argv=None):
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    if args.suite_only:
+        # profiling case: the per-operation figures of the other workloads
+        # only, every count divided by --suite-scale
+        import torch
+        torch.cuda.set_device(0)
+        print(json.dumps({"workloads": workload_suite(torch.device("cuda", 0), peaks()[0],
+                                                      reps=args.steps, scale=args.suite_scale),
+                          "note": "PROFILING CASE, counts / %d" % args.suite_scale}), flush=True)
+        return 0
     if args.impl == "reference":
         res = run_reference(args, rank)
         if res is not None:

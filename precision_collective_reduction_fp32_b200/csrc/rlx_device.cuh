@@ -301,11 +301,11 @@ __device__ __forceinline__ float2 add2_rn(float2 a, float2 b) {
 #endif
 }
 
-// Quantise 4 values of a block with scale sc: code = e4m3_rne_sat(fl32(v/s));
-// s == 0 gives signed zeros.  sc.y == 0 selects the IEEE division.
-__device__ __forceinline__ uint32_t quant4(const float (&v)[4], Scale sc) {
-    float q[4];
-    if (sc.y != 0.0f) {
+// q = fl32(v/s) for 4 values of a block with scale sc; s == 0 gives signed
+// zeros, sc.y == 0 selects the IEEE division.  Fast: sc.y != 0 is known.
+template <bool Fast>
+__device__ __forceinline__ void quotients4(const float (&v)[4], Scale sc, float (&q)[4]) {
+    if (Fast || sc.y != 0.0f) {
         const float2 a = quotient_rn2(f2(v[0], v[1]), sc.s, sc.y);
         const float2 b = quotient_rn2(f2(v[2], v[3]), sc.s, sc.y);
         q[0] = a.x; q[1] = a.y; q[2] = b.x; q[3] = b.y;
@@ -316,14 +316,12 @@ __device__ __forceinline__ uint32_t quant4(const float (&v)[4], Scale sc) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) q[k] = __fdiv_rn(v[k], sc.s);
     }
-    return e4m3x4_from_f32(q);
 }
 
-// quant4 for a block whose scale takes the fast quotient (sc.y != 0).
-__device__ __forceinline__ uint32_t quant4_fast(const float (&v)[4], Scale sc) {
-    const float2 a = quotient_rn2(f2(v[0], v[1]), sc.s, sc.y);
-    const float2 b = quotient_rn2(f2(v[2], v[3]), sc.s, sc.y);
-    const float q[4] = {a.x, a.y, b.x, b.y};
+// Quantise 4 values of a block with scale sc: code = e4m3_rne_sat(fl32(v/s)).
+__device__ __forceinline__ uint32_t quant4(const float (&v)[4], Scale sc) {
+    float q[4];
+    quotients4<false>(v, sc, q);
     return e4m3x4_from_f32(q);
 }
 
@@ -339,6 +337,21 @@ __device__ __forceinline__ void dequant4(uint32_t codes, float s, float (&y)[4])
     y[2] = __fmul_rn(b.x, s); y[3] = __fmul_rn(b.y, s);
 }
 
+// dequantise(quantise(v)) of 4 values of a block, in place: the same steps
+// as dequant4(quant4(v, sc), sc.s, v), with each pair of codes going straight
+// from one conversion to the other instead of through a packed word.
+template <bool Fast>
+__device__ __forceinline__ void wire4(float (&v)[4], Scale sc) {
+    float q[4];
+    quotients4<Fast>(v, sc, q);
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+        const float2 w = e4m3x2_to_f32(e4m3x2_from_f32(q[2 * p], q[2 * p + 1]));
+        v[2 * p] = __fmul_rn(w.x, sc.s);
+        v[2 * p + 1] = __fmul_rn(w.y, sc.s);
+    }
+}
+
 // What a receiver holds after K 128-blocks crossed the FP8 wire.  The warp
 // holds block k as 4 values per lane in v[k] (lanes past a block's end hold
 // +0, which leaves its amax unchanged).  In place.
@@ -350,7 +363,7 @@ __device__ __forceinline__ void wire_fp8_blocks(float (&v)[K][4]) {
     Scale sc[K];
     make_scales<K>(amax, sc);
 #pragma unroll
-    for (int k = 0; k < K; ++k) dequant4(quant4(v[k], sc[k]), sc[k].s, v[k]);
+    for (int k = 0; k < K; ++k) wire4<false>(v[k], sc[k]);
 }
 
 // ----------------------------------------------------------- work layout

@@ -167,7 +167,7 @@ __device__ __forceinline__ void reduce_blocks_fp8(const T *src, size_t pitch, in
                     sc.y = __shfl_sync(kFull, own.y, s * BPU + j);
                     float v[4];
                     widen4(x[s][j], v);
-                    dequant4(decltype(fast)::value ? quant4_fast(v, sc) : quant4(v, sc), sc.s, v);
+                    wire4<decltype(fast)::value>(v, sc);
                     if (s == 0) {
 #pragma unroll
                         for (int k = 0; k < 4; ++k) acc[j][k] = v[k];

@@ -115,18 +115,20 @@ def rank_buffers(workload: int, count: int | None = None, nranks: int | None = N
     return out
 
 
-def device_rank_buffers(workload: int, device, salt: int = 0) -> torch.Tensor:
+def device_rank_buffers(workload: int, device, salt: int = 0,
+                        count: int | None = None) -> torch.Tensor:
     """[nranks, count] torch tensor of a workload drawn directly on a CUDA
     device (fp32, or bf16 rounded from fp32), for timing at full size where
     the host draw would take a minute.  Same recipe as rank_buffers, drawn
     from the device's generator seeded with seed(workload, rank) + salt, so
     the values follow the same distribution but are not the host bytes."""
     w = WORKLOADS[workload]
-    out = torch.empty((w.nranks, w.count), dtype=torch.float32 if w.dtype == "f32"
+    count = w.count if count is None else count
+    out = torch.empty((w.nranks, count), dtype=torch.float32 if w.dtype == "f32"
                       else torch.bfloat16, device=device)
     for r in range(w.nranks):
         g = torch.Generator(device=device).manual_seed(seed(workload, r) + salt)
-        out[r].copy_(_draw(w.dist, w.count, g, w.std, device))
+        out[r].copy_(_draw(w.dist, count, g, w.std, device))
     return out
 
 
