@@ -520,15 +520,20 @@ def _timed_us(call, stream, reps: int, warmup: int = 3) -> float:
     return e0.elapsed_time(e1) / reps * 1e3
 
 
-def _cold_us(call, stream, flush, reps: int) -> float:
-    """Median microseconds of one call with the L2 flushed before it (a
-    write of a buffer larger than L2 between calls, outside the events)."""
+def _cold_us(call, stream, flush, reps: int, dirty: bool = True) -> float:
+    """Median microseconds of one call with the L2 flushed before it, outside
+    the events: by writing a buffer larger than L2 (dirty: the call's misses
+    also evict lines that must be written back) or by reading one (clean)."""
     import torch
     call()
     torch.cuda.synchronize()
     ts = []
+    sink = torch.empty((), dtype=torch.int64, device=flush.device)
     for _ in range(reps):
-        flush.zero_()
+        if dirty:
+            flush.zero_()
+        else:
+            torch.sum(flush, dim=0, dtype=torch.int64, out=sink)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         call()
@@ -541,7 +546,7 @@ def _cold_us(call, stream, flush, reps: int) -> float:
 def workload_suite(dev, peak: float, reps: int = 20, scale: int = 1) -> dict:
     """Per-operation figures on the other full-size workloads, drawn on the
     device (same recipes as the host draws): decode bf16 [32, 8192] x 8 with
-    the L2 cold, prefill bf16 [4096, 8192] x 8 (DDA-tree and -flat, both
+    the L2 cold (flushed by a write, and by a read), prefill bf16 [4096, 8192] x 8 (DDA-tree and -flat, both
     wires) and lp-collectives fp32 [67,108,864] x 8 (reduce-scatter,
     all-gather, alltoall and quantise, both wires)."""
     import torch
@@ -560,7 +565,7 @@ def workload_suite(dev, peak: float, reps: int = 20, scale: int = 1) -> dict:
         return {"us": round(us, 2), "GB/s": round(gbs, 1), "frac": round(gbs / peak, 3),
                 "MiB": round(nbytes / MIB, 2), "floor_us": round(nbytes / (peak * 1e9) * 1e6, 2)}
 
-    def allreduces(x, dcode, esize, cold=None):
+    def allreduces(x, dcode, esize, cold=None, dirty=True):
         n, c = x.shape
         out = torch.empty_like(x)
         ws = torch.empty(max(B.rlx_workspace_bytes(B.RLX_COLL_ALLREDUCE_TREE, c, n, dcode, FP8), 16),
@@ -577,7 +582,7 @@ def workload_suite(dev, peak: float, reps: int = 20, scale: int = 1) -> dict:
                                                             dcode, w, SUM, ws.data_ptr(),
                                                             ws.numel(), sp)
                 nb = ob["allreduce_%s_%s" % (algo, wname)]
-                us = _cold_us(f, st, cold, reps) if cold is not None else _timed_us(f, st, reps)
+                us = _cold_us(f, st, cold, reps, dirty) if cold is not None else _timed_us(f, st, reps)
                 row["allreduce_%s_%s" % (algo, wname)] = entry(us, nb)
         del out, ws
         return row
@@ -586,6 +591,8 @@ def workload_suite(dev, peak: float, reps: int = 20, scale: int = 1) -> dict:
     flush = torch.empty(256 * MIB, dtype=torch.uint8, device=dev)
     x = draw(2)
     res["decode_bf16_8x32x8192_cold_l2"] = allreduces(x, B.RLX_BF16, 2, cold=flush)
+    res["decode_bf16_8x32x8192_cold_l2_clean"] = allreduces(x, B.RLX_BF16, 2, cold=flush,
+                                                           dirty=False)
     del x, flush
     # prefill
     x = draw(3)
