@@ -438,6 +438,24 @@ __device__ __forceinline__ void with_full(bool full, F &&f) {
     else f(std::false_type{});
 }
 
+// The number of ranks a reducing kernel sums, as the compile-time NR when the
+// call uses every rank slot of the kernel (the usual case: N = 2, 4, 8, 16),
+// which removes the per-rank guards, else as a run-time count.
+struct RankCount {
+    int v;
+    __device__ __forceinline__ operator int() const { return v; }
+};
+template <int NR> struct FixedRanks {
+    __device__ __forceinline__ constexpr operator int() const { return NR; }
+};
+// EXACT (n == NR) is chosen by the host, so each kernel instantiation holds
+// one of the two forms and keeps its registers to itself.
+template <int NR, bool EXACT, typename F>
+__device__ __forceinline__ void with_rank_count(int n, F &&f) {
+    if constexpr (EXACT) f(FixedRanks<NR>{});
+    else f(RankCount{n});
+}
+
 // Calls f(std::true_type{}) when every block scale of the unit takes the fast
 // quotient, else f(std::false_type{}).
 template <typename F>

@@ -86,8 +86,8 @@ __device__ __forceinline__ void add_raw(float (&acc)[VecN<T>::n], const uint4 &q
 // of the n rows (row pitch `pitch` elements).  Full vectors issue all n loads
 // before the first add; a partial (tail) vector is summed rank by rank, which
 // needs few registers and keeps the kernel's register budget for the hot path.
-template <typename T, int NR, bool VEC, typename Full>
-__device__ __forceinline__ void reduce_vec(const T *src, size_t pitch, int n, int valid, Full,
+template <typename T, int NR, bool VEC, typename Full, typename N>
+__device__ __forceinline__ void reduce_vec(const T *src, size_t pitch, N n, int valid, Full,
                                            float (&acc)[VecN<T>::n]) {
     if constexpr (Full::value) {
         uint4 x[NR];
@@ -129,8 +129,8 @@ template <typename T> constexpr int kBpu = sizeof(T) == 2 ? RLX_BPU_BF16 : 1;
 // reduction, and lane l computes the scale of pair l % (NR*BPU), which is
 // broadcast just before that pair is quantised.  The loads stay raw until
 // then, so a bf16 pair costs 2 registers.
-template <typename T, int NR, bool VEC, int BPU>
-__device__ __forceinline__ void reduce_blocks_fp8(const T *src, size_t pitch, int n,
+template <typename T, int NR, bool VEC, int BPU, typename N>
+__device__ __forceinline__ void reduce_blocks_fp8(const T *src, size_t pitch, N n,
                                                   const int (&valid)[BPU],
                                                   float (&acc)[BPU][4]) {
     constexpr int K = NR * BPU;
@@ -216,8 +216,8 @@ __device__ __forceinline__ bool rows_16b(const T *p, size_t pitch) {
 // Stores the reduced blocks of a unit (acc[j] = block j, 4 values per lane) at
 // dst + 128 j in each of `rows` rows `pitch` apart.  A full bf16 block pair
 // on 16-byte aligned rows goes out as 16-byte pieces.
-template <typename T, bool VEC, int BPU, typename Full>
-__device__ __forceinline__ void store_blocks(T *dst, size_t pitch, int rows, Full, bool wide,
+template <typename T, bool VEC, int BPU, typename Full, typename R>
+__device__ __forceinline__ void store_blocks(T *dst, size_t pitch, R rows, Full, bool wide,
                                              const int (&valid)[BPU], const float (&acc)[BPU][4]) {
     if constexpr (BPU == 2 && sizeof(T) == 2 && Full::value) {
         if (VEC && wide) {
@@ -357,9 +357,9 @@ __device__ __forceinline__ bool unit_full(size_t unit, size_t len) {
 // ------------------------------------------------------ DDA-tree pass units
 
 // Pass 1, native: unit g = (chunk c, 32 vectors of it); chunk c -> row c.
-template <typename T, int NR, bool VEC>
+template <typename T, int NR, bool VEC, typename N>
 __device__ __forceinline__ void tree_reduce_native_unit(uint32_t g, const T *send, T *recv,
-                                                        size_t count, size_t stride, int n,
+                                                        size_t count, size_t stride, N n,
                                                         size_t chunk, const FastDiv &per_chunk) {
     constexpr int V = VecN<T>::n;
     const uint32_t c = fast_div(g, per_chunk);
@@ -380,9 +380,9 @@ __device__ __forceinline__ void tree_reduce_native_unit(uint32_t g, const T *sen
 // Pass 1, FP8: unit u = the BPU blocks from block u*BPU on; reduce, then
 // quantise each reduced block again into the payload (codes padded to whole
 // blocks, one scale per block).
-template <typename T, int NR, bool VEC>
+template <typename T, int NR, bool VEC, typename N>
 __device__ __forceinline__ void tree_reduce_fp8_unit(uint32_t u, const T *send, size_t count,
-                                                     size_t stride, int n, uint8_t *ws_codes,
+                                                     size_t stride, N n, uint8_t *ws_codes,
                                                      float *ws_scales) {
     constexpr int BPU = kBpu<T>;
     const int e0 = lane_id() * 4;

@@ -69,121 +69,143 @@ constexpr int kMinBlocksFp8 = NR > 8 ? 1 : sizeof(T) == 2 ? RLX_MINB_FP8_BF16 : 
 template <int NR> constexpr int kMinBlocksFp8Flat = NR <= 8 ? RLX_MINB_FP8_FLAT : 1;
 
 // DDA-flat, native: unit g = 32 consecutive 16-byte vectors (lane l: 32g + l).
-template <typename T, int NR, bool VEC>
+template <typename T, int NR, bool VEC, bool EXACT>
 __global__ void __launch_bounds__(kThreads, kMinBlocksNative<NR>)
 flat_native_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
     constexpr int V = VecN<T>::n;
     const size_t nvec = (count + V - 1) / V;
     const uint32_t units = static_cast<uint32_t>((nvec + 31) / 32);
-    for_each_unit<kPn>(units, [&](uint32_t g) {
-        const size_t i0 = (static_cast<size_t>(g) * 32 + lane_id()) * V;
-        with_full((static_cast<size_t>(g) + 1) * 32 * V <= count, [&](auto full) {
-            const int valid = vec_valid_in<V>(i0, count, full);
-            if (valid == 0) return;
-            float acc[V];
-            reduce_vec<T, NR, VEC>(send + i0, stride, n, valid, full, acc);
-            for (int r = 0; r < n; ++r) storev<T, VEC>(recv + r * stride + i0, valid, acc);
+    with_rank_count<NR, EXACT>(n, [&](auto nn) {
+        for_each_unit<kPn>(units, [&](uint32_t g) {
+            const size_t i0 = (static_cast<size_t>(g) * 32 + lane_id()) * V;
+            with_full((static_cast<size_t>(g) + 1) * 32 * V <= count, [&](auto full) {
+                const int valid = vec_valid_in<V>(i0, count, full);
+                if (valid == 0) return;
+                float acc[V];
+                reduce_vec<T, NR, VEC>(send + i0, stride, nn, valid, full, acc);
+                for (int r = 0; r < nn; ++r) storev<T, VEC>(recv + r * stride + i0, valid, acc);
+            });
         });
     });
 }
 
 // DDA-flat, FP8: unit u = the kBpu<T> blocks from block u*kBpu<T> on.
-template <typename T, int NR, bool VEC>
+template <typename T, int NR, bool VEC, bool EXACT>
 __global__ void __launch_bounds__(kThreads, kMinBlocksFp8Flat<NR>)
 flat_fp8_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
     constexpr int BPU = kBpu<T>;
     const uint32_t units = static_cast<uint32_t>((count + BPU * kBlock - 1) / (BPU * kBlock));
     const bool wide = rows_16b(recv, stride);
-    for_each_unit<kPfFlat>(units, [&](uint32_t u) {
-        const size_t base = static_cast<size_t>(u) * BPU * kBlock;
-        with_full(base + BPU * kBlock <= count, [&](auto full) {
-            int valid[BPU];
+    with_rank_count<NR, EXACT>(n, [&](auto nn) {
+        for_each_unit<kPfFlat>(units, [&](uint32_t u) {
+            const size_t base = static_cast<size_t>(u) * BPU * kBlock;
+            with_full(base + BPU * kBlock <= count, [&](auto full) {
+                int valid[BPU];
 #pragma unroll
-            for (int j = 0; j < BPU; ++j)
-                valid[j] = decltype(full)::value ? 4 : lane_valid(base + j * kBlock, count);
-            float acc[BPU][4];
-            reduce_blocks_fp8<T, NR, VEC, BPU>(send + base, stride, n, valid, acc);
-            store_blocks<T, VEC, BPU>(recv + base, stride, n, full, wide, valid, acc);
+                for (int j = 0; j < BPU; ++j)
+                    valid[j] = decltype(full)::value ? 4 : lane_valid(base + j * kBlock, count);
+                float acc[BPU][4];
+                reduce_blocks_fp8<T, NR, VEC, BPU>(send + base, stride, nn, valid, acc);
+                store_blocks<T, VEC, BPU>(recv + base, stride, nn, full, wide, valid, acc);
+            });
         });
     });
 }
 
 // DDA-tree pass 1, native (one unit body per unit, see rlx_passes.cuh).
-template <typename T, int NR, bool VEC>
+template <typename T, int NR, bool VEC, bool EXACT>
 __global__ void __launch_bounds__(kThreads, kMinBlocksNative<NR>)
 tree_reduce_native_kernel(const T *send, T *recv, size_t count, size_t stride, int n,
                           size_t chunk, FastDiv per_chunk) {
     const uint32_t units = per_chunk.d * static_cast<uint32_t>(n);
-    for_each_unit<kPn>(units, [&](uint32_t g) {
-        tree_reduce_native_unit<T, NR, VEC>(g, send, recv, count, stride, n, chunk, per_chunk);
+    with_rank_count<NR, EXACT>(n, [&](auto nn) {
+        for_each_unit<kPn>(units, [&](uint32_t g) {
+            tree_reduce_native_unit<T, NR, VEC>(g, send, recv, count, stride, nn, chunk, per_chunk);
+        });
     });
 }
 
 // DDA-tree pass 1, FP8.
-template <typename T, int NR, bool VEC, int P>
+template <typename T, int NR, bool VEC, int P, bool EXACT>
 __global__ void __launch_bounds__(kThreads, kMinBlocksFp8<T, NR>)
 tree_reduce_fp8_kernel(const T *send, size_t count, size_t stride, int n,
                        uint8_t *ws_codes, float *ws_scales) {
     constexpr int BPU = kBpu<T>;
     const uint32_t units = static_cast<uint32_t>((count + BPU * kBlock - 1) / (BPU * kBlock));
-    for_each_unit<P>(units, [&](uint32_t u) {
-        tree_reduce_fp8_unit<T, NR, VEC>(u, send, count, stride, n, ws_codes, ws_scales);
+    with_rank_count<NR, EXACT>(n, [&](auto nn) {
+        for_each_unit<P>(units, [&](uint32_t u) {
+            tree_reduce_fp8_unit<T, NR, VEC>(u, send, count, stride, nn, ws_codes, ws_scales);
+        });
     });
 }
 
 // ReduceScatter, native: unit = (destination rank r, 32 vectors of chunk r).
-template <typename T, int NR, bool VEC>
+template <typename T, int NR, bool VEC, bool EXACT>
 __global__ void __launch_bounds__(kThreads, kMinBlocksNative<NR>)
 rs_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n,
                  FastDiv per_chunk) {
     constexpr int V = VecN<T>::n;
     const uint32_t units = per_chunk.d * static_cast<uint32_t>(n);
-    for_each_unit<kPn>(units, [&](uint32_t g) {
-        const uint32_t r = fast_div(g, per_chunk);
-        const size_t u0 = static_cast<size_t>(g - r * per_chunk.d) * 32 * V;
-        const size_t j0 = u0 + static_cast<size_t>(lane_id()) * V;
-        with_full(u0 + 32 * V <= m, [&](auto full) {
-            const int valid = vec_valid_in<V>(j0, m, full);
-            if (valid == 0) return;
-            float acc[V];
-            reduce_vec<T, NR, VEC>(send + r * m + j0, sstride, n, valid, full, acc);
-            storev<T, VEC>(recv + r * rstride + j0, valid, acc);
+    with_rank_count<NR, EXACT>(n, [&](auto nn) {
+        for_each_unit<kPn>(units, [&](uint32_t g) {
+            const uint32_t r = fast_div(g, per_chunk);
+            const size_t u0 = static_cast<size_t>(g - r * per_chunk.d) * 32 * V;
+            const size_t j0 = u0 + static_cast<size_t>(lane_id()) * V;
+            with_full(u0 + 32 * V <= m, [&](auto full) {
+                const int valid = vec_valid_in<V>(j0, m, full);
+                if (valid == 0) return;
+                float acc[V];
+                reduce_vec<T, NR, VEC>(send + r * m + j0, sstride, nn, valid, full, acc);
+                storev<T, VEC>(recv + r * rstride + j0, valid, acc);
+            });
         });
     });
 }
 
 // ReduceScatter, FP8: unit = (destination rank r, kBpu<T> adjacent blocks of
 // chunk r); blocks anchored at the chunk start r*m.
-template <typename T, int NR, bool VEC, int P>
+template <typename T, int NR, bool VEC, int P, bool EXACT>
 __global__ void __launch_bounds__(kThreads, kMinBlocksFp8<T, NR>)
 rs_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n,
               FastDiv per_chunk) {
     constexpr int BPU = kBpu<T>;
     const uint32_t units = per_chunk.d * static_cast<uint32_t>(n);
     const bool wide = rows_16b(recv, rstride);
-    for_each_unit<P>(units, [&](uint32_t g) {
-        const uint32_t r = fast_div(g, per_chunk);
-        const size_t j0 = static_cast<size_t>(g - r * per_chunk.d) * BPU * kBlock;
-        with_full(j0 + BPU * kBlock <= m, [&](auto full) {
-            int valid[BPU];
+    with_rank_count<NR, EXACT>(n, [&](auto nn) {
+        for_each_unit<P>(units, [&](uint32_t g) {
+            const uint32_t r = fast_div(g, per_chunk);
+            const size_t j0 = static_cast<size_t>(g - r * per_chunk.d) * BPU * kBlock;
+            with_full(j0 + BPU * kBlock <= m, [&](auto full) {
+                int valid[BPU];
 #pragma unroll
-            for (int j = 0; j < BPU; ++j)
-                valid[j] = decltype(full)::value ? 4 : lane_valid(j0 + j * kBlock, m);
-            float acc[BPU][4];
-            reduce_blocks_fp8<T, NR, VEC, BPU>(send + r * m + j0, sstride, n, valid, acc);
-            store_blocks<T, VEC, BPU>(recv + r * rstride + j0, rstride, 1, full, wide, valid, acc);
+                for (int j = 0; j < BPU; ++j)
+                    valid[j] = decltype(full)::value ? 4 : lane_valid(j0 + j * kBlock, m);
+                float acc[BPU][4];
+                reduce_blocks_fp8<T, NR, VEC, BPU>(send + r * m + j0, sstride, nn, valid, acc);
+                store_blocks<T, VEC, BPU>(recv + r * rstride + j0, rstride, 1, full, wide, valid,
+                                          acc);
+            });
         });
     });
 }
 
 // ------------------------------------------------------------- dispatching
 
-// Calls f.template operator()<T, NR, VEC>() for the rank bound NR >= n.
+// Calls f.template operator()<T, NR, VEC, EX>() for the rank bound NR >= n;
+// EX: n == NR (the kernel sums a compile-time number of ranks).
+#ifndef RLX_FIXED_RANKS
+#define RLX_FIXED_RANKS 1
+#endif
+template <typename T, int NRV, bool VEC, typename F>
+cudaError_t dispatch_exact(int n, F &&f) {
+    if (RLX_FIXED_RANKS && n == NRV) return f.template operator()<T, NRV, VEC, true>();
+    return f.template operator()<T, NRV, VEC, false>();
+}
 template <typename F>
 cudaError_t dispatch(rlx_dtype dtype, int n, bool vec, F &&f) {
 #define RLX_CASE_NR(T, NRV)                                                       \
-    if (n <= NRV) return vec ? f.template operator()<T, NRV, true>()              \
-                             : f.template operator()<T, NRV, false>();
+    if (n <= NRV) return vec ? dispatch_exact<T, NRV, true>(n, f)                 \
+                             : dispatch_exact<T, NRV, false>(n, f);
 #define RLX_CASE_T(T) \
     RLX_CASE_NR(T, 2) RLX_CASE_NR(T, 4) RLX_CASE_NR(T, 8) RLX_CASE_NR(T, 16)
     if (dtype == RLX_F32) { RLX_CASE_T(float) }
@@ -208,16 +230,18 @@ constexpr size_t kWarps = kThreads / 32;
 cudaError_t launch_allreduce_flat(const void *send, void *recv, size_t count, size_t stride,
                                   int nranks, rlx_dtype dtype, rlx_wire wire, bool vec,
                                   cudaStream_t stream) {
-    return dispatch(dtype, nranks, vec, [&]<typename T, int NR, bool VEC>() {
+    return dispatch(dtype, nranks, vec, [&]<typename T, int NR, bool VEC, bool EX>() {
         const T *s = static_cast<const T *>(send);
         T *r = static_cast<T *>(recv);
         if (wire == RLX_WIRE_NATIVE) {
+            // the run-time rank count measured faster here than the compile-time
+            // one (159.5 against 161.9 us at 8 x 16 Mi fp32)
             const size_t units = ((count + VecN<T>::n - 1) / VecN<T>::n + 31) / 32;
-            return launch(flat_native_kernel<T, NR, VEC>, units, kWarps * kPn, stream, s, r,
+            return launch(flat_native_kernel<T, NR, VEC, false>, units, kWarps * kPn, stream, s, r,
                           count, stride, nranks);
         }
         const size_t units = (count + kBpu<T> * kBlock - 1) / (kBpu<T> * kBlock);
-        return launch(flat_fp8_kernel<T, NR, VEC>, units, kWarps * kPfFlat, stream, s, r, count,
+        return launch(flat_fp8_kernel<T, NR, VEC, EX>, units, kWarps * kPfFlat, stream, s, r, count,
                       stride, nranks);
     });
 }
@@ -226,12 +250,12 @@ cudaError_t launch_tree_reduce(const void *send, void *recv, size_t count, size_
                                int nranks, size_t chunk, rlx_dtype dtype, rlx_wire wire,
                                uint8_t *ws_codes, float *ws_scales, bool vec,
                                cudaStream_t stream) {
-    return dispatch(dtype, nranks, vec, [&]<typename T, int NR, bool VEC>() {
+    return dispatch(dtype, nranks, vec, [&]<typename T, int NR, bool VEC, bool EX>() {
         const T *s = static_cast<const T *>(send);
         if (wire == RLX_WIRE_NATIVE) {
             const size_t per = tree_reduce_native_per_chunk<T>(chunk);
             if (per >= (size_t{1} << 32)) return cudaErrorInvalidValue;
-            return launch(tree_reduce_native_kernel<T, NR, VEC>,
+            return launch(tree_reduce_native_kernel<T, NR, VEC, EX>,
                           per * static_cast<size_t>(nranks), kWarps * kPn, stream, s,
                           static_cast<T *>(recv), count, stride, nranks, chunk,
                           make_fastdiv(static_cast<uint32_t>(per)));
@@ -239,9 +263,9 @@ cudaError_t launch_tree_reduce(const void *send, void *recv, size_t count, size_
         const size_t nblk = (count + kBlock - 1) / kBlock;
         const size_t units = (nblk + kBpu<T> - 1) / kBpu<T>;
         if (nblk < RLX_FP8_SMALL_BLOCKS)
-            return launch(tree_reduce_fp8_kernel<T, NR, VEC, 1>, units, kWarps, stream, s, count,
+            return launch(tree_reduce_fp8_kernel<T, NR, VEC, 1, EX>, units, kWarps, stream, s, count,
                           stride, nranks, ws_codes, ws_scales);
-        return launch(tree_reduce_fp8_kernel<T, NR, VEC, kPf>, units, kWarps * kPf, stream, s,
+        return launch(tree_reduce_fp8_kernel<T, NR, VEC, kPf, EX>, units, kWarps * kPf, stream, s,
                       count, stride, nranks, ws_codes, ws_scales);
     });
 }
@@ -249,7 +273,7 @@ cudaError_t launch_tree_reduce(const void *send, void *recv, size_t count, size_
 cudaError_t launch_reduce_scatter(const void *send, size_t send_stride, void *recv,
                                   size_t recv_stride, size_t m, int nranks, rlx_dtype dtype,
                                   rlx_wire wire, bool vec, cudaStream_t stream) {
-    return dispatch(dtype, nranks, vec, [&]<typename T, int NR, bool VEC>() {
+    return dispatch(dtype, nranks, vec, [&]<typename T, int NR, bool VEC, bool EX>() {
         const T *s = static_cast<const T *>(send);
         T *r = static_cast<T *>(recv);
         const size_t nn = static_cast<size_t>(nranks);
@@ -259,12 +283,12 @@ cudaError_t launch_reduce_scatter(const void *send, size_t send_stride, void *re
         if (per >= (size_t{1} << 32)) return cudaErrorInvalidValue;
         const FastDiv fd = make_fastdiv(static_cast<uint32_t>(per));
         if (wire == RLX_WIRE_NATIVE)
-            return launch(rs_native_kernel<T, NR, VEC>, per * nn, kWarps * kPn, stream, s,
+            return launch(rs_native_kernel<T, NR, VEC, EX>, per * nn, kWarps * kPn, stream, s,
                           send_stride, r, recv_stride, m, nranks, fd);
         if (per * kBpu<T> * nn < RLX_FP8_SMALL_BLOCKS)
-            return launch(rs_fp8_kernel<T, NR, VEC, 1>, per * nn, kWarps, stream, s, send_stride,
+            return launch(rs_fp8_kernel<T, NR, VEC, 1, EX>, per * nn, kWarps, stream, s, send_stride,
                           r, recv_stride, m, nranks, fd);
-        return launch(rs_fp8_kernel<T, NR, VEC, kPf>, per * nn, kWarps * kPf, stream, s,
+        return launch(rs_fp8_kernel<T, NR, VEC, kPf, EX>, per * nn, kWarps * kPf, stream, s,
                       send_stride, r, recv_stride, m, nranks, fd);
     });
 }
