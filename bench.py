@@ -546,9 +546,10 @@ def _cold_us(call, stream, flush, reps: int, dirty: bool = True) -> float:
 def workload_suite(dev, peak: float, reps: int = 20, scale: int = 1) -> dict:
     """Per-operation figures on the other full-size workloads, drawn on the
     device (same recipes as the host draws): decode bf16 [32, 8192] x 8 with
-    the L2 cold (flushed by a write, and by a read), prefill bf16 [4096, 8192] x 8 (DDA-tree and -flat, both
-    wires) and lp-collectives fp32 [67,108,864] x 8 (reduce-scatter,
-    all-gather, alltoall and quantise, both wires)."""
+    the L2 cold (flushed by a write, and by a read), prefill bf16 [4096, 8192]
+    x 8 (DDA-tree and -flat, reduce-scatter, all-gather, alltoall, both wires)
+    and lp-collectives fp32 [67,108,864] x 8 (quantise, reduce-scatter,
+    all-gather, alltoall, both wires)."""
     import torch
     from precision_collective_reduction_fp32_b200 import binding as B
     from precision_collective_reduction_fp32_b200 import synth
@@ -587,6 +588,34 @@ def workload_suite(dev, peak: float, reps: int = 20, scale: int = 1) -> dict:
         del out, ws
         return row
 
+    def chunked(x, dcode, esize, quantise):
+        """quantise (optional), reduce-scatter, all-gather of its result and
+        alltoall of x, both wires, on [N, c] rank buffers x."""
+        n, c = x.shape
+        m = c // n
+        ob = op_bytes(c, n, esize)
+        y = torch.empty_like(x)
+        rs = torch.empty((n, m), dtype=x.dtype, device=dev)
+        row = {}
+        if quantise:
+            codes = torch.empty((n, c), dtype=torch.uint8, device=dev)
+            scales = torch.empty((n, (c + BLOCK - 1) // BLOCK), dtype=torch.float32, device=dev)
+            row["quantize_fp8"] = entry(_timed_us(lambda: B.rlx_quantize_fp8(
+                x.data_ptr(), dcode, n, c, c, codes.data_ptr(), scales.data_ptr(), sp), st, reps),
+                ob["quantize_fp8"])
+            del codes, scales
+        for wname, wire in wires:
+            row["reduce_scatter_" + wname] = entry(_timed_us(lambda: B.rlx_reduce_scatter(
+                x.data_ptr(), c, rs.data_ptr(), m, m, n, dcode, wire, SUM, sp), st, reps),
+                ob["reduce_scatter_" + wname])
+            row["all_gather_" + wname] = entry(_timed_us(lambda: B.rlx_all_gather(
+                rs.data_ptr(), m, y.data_ptr(), c, m, n, dcode, wire, sp), st, reps),
+                ob["all_gather_" + wname])
+            row["alltoall_" + wname] = entry(_timed_us(lambda: B.rlx_alltoall(
+                x.data_ptr(), c, y.data_ptr(), c, m, n, dcode, wire, sp), st, reps),
+                ob["alltoall_" + wname])
+        return row
+
     # decode, L2 cold (the hot-L2 figures are under small_messages)
     flush = torch.empty(256 * MIB, dtype=torch.uint8, device=dev)
     x = draw(2)
@@ -594,36 +623,15 @@ def workload_suite(dev, peak: float, reps: int = 20, scale: int = 1) -> dict:
     res["decode_bf16_8x32x8192_cold_l2_clean"] = allreduces(x, B.RLX_BF16, 2, cold=flush,
                                                            dirty=False)
     del x, flush
-    # prefill
+    # prefill, and the chunked collectives on the same bf16 rank buffers
     x = draw(3)
     res["prefill_bf16_8x4096x8192"] = allreduces(x, B.RLX_BF16, 2)
+    res["prefill_bf16_8x4096x8192"].update(chunked(x, B.RLX_BF16, 2, quantise=False))
     del x
     # lp-collectives
     x = draw(5)
-    n, c = x.shape
-    m = c // n
-    ob = op_bytes(c, n)
-    y = torch.empty_like(x)
-    rs = torch.empty((n, m), dtype=torch.float32, device=dev)
-    codes = torch.empty((n, c), dtype=torch.uint8, device=dev)
-    scales = torch.empty((n, (c + BLOCK - 1) // BLOCK), dtype=torch.float32, device=dev)
-    F = B.RLX_F32
-    row = {}
-    row["quantize_fp8"] = entry(_timed_us(lambda: B.rlx_quantize_fp8(
-        x.data_ptr(), F, n, c, c, codes.data_ptr(), scales.data_ptr(), sp), st, reps),
-        ob["quantize_fp8"])
-    for wname, wire in wires:
-        row["reduce_scatter_" + wname] = entry(_timed_us(lambda: B.rlx_reduce_scatter(
-            x.data_ptr(), c, rs.data_ptr(), m, m, n, F, wire, SUM, sp), st, reps),
-            ob["reduce_scatter_" + wname])
-        row["all_gather_" + wname] = entry(_timed_us(lambda: B.rlx_all_gather(
-            rs.data_ptr(), m, y.data_ptr(), c, m, n, F, wire, sp), st, reps),
-            ob["all_gather_" + wname])
-        row["alltoall_" + wname] = entry(_timed_us(lambda: B.rlx_alltoall(
-            x.data_ptr(), c, y.data_ptr(), c, m, n, F, wire, sp), st, reps),
-            ob["alltoall_" + wname])
-    res["lp_collectives_fp32_8x67108864"] = row
-    del x, y, rs, codes, scales
+    res["lp_collectives_fp32_8x67108864"] = chunked(x, B.RLX_F32, 4, quantise=True)
+    del x
     torch.cuda.empty_cache()
     return res
 

@@ -337,6 +337,25 @@ def test_alltoall(wire, dtype, nranks, m):
         assert _bits_equal(got, ref), (pad, off)
 
 
+@pytest.mark.parametrize("name", ["rlx_all_gather", "rlx_alltoall"])
+@pytest.mark.parametrize("m", [8192 + 256, 3 * 1024 + 8])
+def test_bf16_fp8_gathers_wide(name, m):
+    """bf16 on the FP8 wire with whole 8-block units and 16-byte aligned rows
+    (block pairs read and written as 16-byte pieces), a ragged last unit, and
+    the same shapes on rows that are not 16-byte aligned."""
+    n = 8
+    for pad, off in ((0, 0), (8, 0), (4, 0), (0, 1)):   # 16-byte, 16-byte, 8-byte, 2-byte rows
+        if name == "rlx_all_gather":
+            x = synth.rank_buffers(5, count=m, nranks=n, stride=m + pad, dtype="bf16")
+            got = _chunked(name, x, m, m + pad, n * m + pad, n * m, B.RLX_WIRE_FP8_E4M3, off)
+            ref = oracle.all_gather(x, m, wire=oracle.FP8, recv_stride=n * m + pad)
+        else:
+            x = synth.rank_buffers(5, count=n * m, nranks=n, stride=n * m + pad, dtype="bf16")
+            got = _chunked(name, x, m, n * m + pad, n * m + pad, n * m, B.RLX_WIRE_FP8_E4M3, off)
+            ref = oracle.alltoall(x, m, wire=oracle.FP8, recv_stride=n * m + pad)
+        assert _bits_equal(got, ref), (pad, off)
+
+
 def test_torch_level_api_matches_c_abi():
     import precision_collective_reduction_fp32_b200 as rlx
     x = synth.rank_buffers(4, count=4096, nranks=8)
