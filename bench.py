@@ -47,6 +47,7 @@ BLOCK = 128
 MIB = 1 << 20
 WORKLOAD = 4        # seeded workload id in synth (N(0,1) + 1% x100 outliers)
 CPU_SAMPLE = 8_388_608   # elements per rank in the oracle's bounded sample (~10 s)
+HBM_NOMINAL_GBS = 7700.0  # B200 HBM3e, nominal (the roofline itself uses the measured copy peak)
 
 
 # --------------------------------------------------------------- bytes model
@@ -378,6 +379,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         ms = per_op_ms[name] / K
         gbs = bytes_[name] / (ms * 1e-3) / 1e9
         per_op[name] = {"us": round(ms * 1e3, 2), "GB/s": round(gbs, 1),
+                        "Gelem/s": round(NRANKS * count / (ms * 1e-3) / 1e9, 1),
                         "frac": round(gbs / peak, 3), "MiB": round(bytes_[name] / MIB, 1)}
     single = [n for n in per_op_ms if KERNELS_PER_OP[n] == 1]
     dom = max(single, key=lambda n: per_op_ms[n])
@@ -408,6 +410,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
             "parallelism": "independent batch per GPU" if world > 1 else "single GPU",
         },
         "hbm_frac": round(value / world / peak, 3),
+        "hbm_frac_nominal": round(value / world / HBM_NOMINAL_GBS, 3),
         "ops": per_op,
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": dom_gbs, "peak": peak,
                      "unit": "GB/s", "frac": round(dom_gbs / peak, 3), "traffic": traffic,
