@@ -150,3 +150,15 @@ def test_binding_raises_without_gpu_work(L):
     with pytest.raises(B.RlxError) as e:
         B.rlx_allreduce_flat(A, A + Z, 100, 99, 8, F32, NAT)
     assert e.value.status == B.RLX_ERR_INVALID_ARG
+
+
+def test_build_flags_keep_ieee_rounding():
+    """Parity with the oracle depends on these: no multiply-add contraction,
+    correctly rounded division and square root, subnormals kept, and code
+    for sm_100a only."""
+    from precision_collective_reduction_fp32_b200 import build
+    f = build.FLAGS
+    for flag in ("-fmad=false", "-prec-div=true", "-prec-sqrt=true", "-ftz=false"):
+        assert flag in f
+    assert "arch=compute_100a,code=sm_100a" in f
+    assert not any(x.startswith("--use_fast_math") or x == "-use_fast_math" for x in f)
