@@ -39,7 +39,9 @@
  * Conventions for every entry point
  *   - Pointers are DEVICE pointers (cudaMalloc / torch CUDA memory) on the
  *     current device; the caller owns every buffer.  The library allocates
- *     nothing and keeps no state between calls.
+ *     nothing.  It keeps no state between calls, with one exception: the
+ *     fixed device array of rlx_allreduce_tree_noalloc and the cache of its
+ *     device address (one entry per device, see that entry point).
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is only
  *     enqueued: the call returns before the GPU finishes.  Faults during the
  *     kernel surface at the caller's next synchronisation.
@@ -190,7 +192,10 @@ RLX_API rlx_status rlx_alltoall(const void *send, size_t send_stride, void *recv
  * and has no such limit.  The library allocates nothing.
  *
  * The first call on each device looks up the array's device address with
- * that device current; make that first call before any stream capture.
+ * that device current and caches it with the id of the device's CUDA
+ * context; after the context is replaced (cudaDeviceReset) the next call
+ * looks the address up again.  Make such a first call before any stream
+ * capture.
  * All calls on a device share the one array: two calls whose kernels can
  * overlap on the GPU (different streams, no ordering between them) race on
  * it.  Calls ordered on one stream are safe; nothing in the array needs to

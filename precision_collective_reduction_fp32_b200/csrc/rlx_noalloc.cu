@@ -12,17 +12,23 @@
 // by pass 1 and read by pass 2) lives in `g_tree_scratch`, a file-scope
 // __device__ array of kScratchBytes, enough for RLX_NOALLOC_MAX_COUNT
 // elements per rank (16 Mi elements: 16.5 MiB).  Every GPU that loads the
-// library holds that array until the process exits.  Host code cannot use the array's name
-// as a device address, so on the first call on each device this file asks
-// the runtime for the address (cudaGetSymbolAddress, with that device
-// current) and caches it; that first call should come before any stream
-// capture.  Every call on a device shares the one array and the array keeps
-// the last call's contents; nothing in it has to start at zero, because pass
-// 1 writes every code and scale of every block before pass 2 reads them.
-// Two calls whose kernels overlap on the GPU (different streams, no
-// ordering between them) race on the array.
+// library holds that array until the process exits.  Host code cannot use
+// the array's name as a device address, so this file asks the runtime for
+// the address (cudaGetSymbolAddress, with the device current) and caches it
+// per device,
+// together with the id of the CUDA context it was taken in.  The lookup
+// happens on the first call on each device, and again on the first call
+// after that device's context was replaced (cudaDeviceReset reloads the
+// module, and the array may then sit elsewhere); such a first call should
+// come before any stream capture.  Every call on a device shares the one
+// array and the array keeps the last call's contents; nothing in it has to
+// start at zero, because pass 1 writes every code and scale of every block
+// before pass 2 reads them.  Two calls whose kernels overlap on the GPU
+// (different streams, no ordering between them) race on the array.
 #include <cstdint>
 #include <mutex>
+
+#include <cuda.h>
 
 #include "rlx_internal.h"
 
@@ -34,11 +40,33 @@ constexpr size_t kScratchBytes =
 __device__ __align__(256) uint8_t g_tree_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
+struct Slot {
+    unsigned long long ctx;   // id of the context the address was taken in (0: none known)
+    void *ptr;
+};
 std::mutex g_mu;
-void *g_scratch_ptr[kMaxDevices] = {};
+Slot g_slot[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device, looked up once
-// per device with that device current.  nullptr (and *err set) on failure.
+// Id of the calling thread's current CUDA context, through the driver's
+// cuCtxGetId fetched from the runtime (no link-time dependency on the driver
+// library).  false when there is no current context or the query fails.
+bool current_context_id(unsigned long long *id) {
+    using GetId = CUresult (*)(CUcontext, unsigned long long *);
+    static GetId fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<GetId>(p);
+    }();
+    return fn != nullptr && fn(nullptr, id) == CUDA_SUCCESS && *id != 0;
+}
+
+// Device address of the scratch array in the current device's context,
+// looked up with that device current on the first call in each context.
+// nullptr (and *err set) on failure.
 void *scratch_address(cudaError_t *err) {
     int dev = 0;
     *err = cudaGetDevice(&dev);
@@ -47,14 +75,19 @@ void *scratch_address(cudaError_t *err) {
         *err = cudaErrorInvalidDevice;
         return nullptr;
     }
+    unsigned long long ctx = 0;
+    const bool known = current_context_id(&ctx);
     std::lock_guard<std::mutex> lock(g_mu);
-    if (g_scratch_ptr[dev] == nullptr) {
+    Slot &slot = g_slot[dev];
+    if (slot.ptr == nullptr || !known || slot.ctx != ctx) {
         void *p = nullptr;
-        *err = cudaGetSymbolAddress(&p, g_tree_scratch);
+        *err = cudaGetSymbolAddress(&p, g_tree_scratch);   // makes the context current too
         if (*err != cudaSuccess) return nullptr;
-        g_scratch_ptr[dev] = p;
+        unsigned long long now = 0;
+        slot.ctx = current_context_id(&now) ? now : 0;     // 0: look up again next call
+        slot.ptr = p;
     }
-    return g_scratch_ptr[dev];
+    return slot.ptr;
 }
 
 }  // namespace

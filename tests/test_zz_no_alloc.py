@@ -7,15 +7,19 @@ different inputs, and compares each result with rlx_allreduce_tree given a
 workspace allocated here -- bit for bit, the bar of every parity test in
 this suite (the arithmetic is the same; only where the payload lives
 differs).  The second call also shows that the payload left behind by the
-first call does not leak into the next result.  This file is collected last
-and works on its own in a fresh process (it builds and loads the library
-itself).
+first call does not leak into the next result.  Two FP8 cases are also
+compared with the CPU oracle's DDA-tree, again on two calls in a row.
+This file is collected last and works on its own in a fresh process (it
+builds and loads the library itself).
 """
+import numpy as np
 import pytest
 import torch
 
+import oracle
 from precision_collective_reduction_fp32_b200 import binding as B
 from precision_collective_reduction_fp32_b200 import build as rlx_build
+from precision_collective_reduction_fp32_b200 import synth
 
 pytestmark = pytest.mark.gpu
 
@@ -32,6 +36,7 @@ CASES = [  # (nranks, count, stride, dtype, wire)
 def _lib():
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
     rlx_build.build()
+    oracle.build()
     B.lib()
 
 
@@ -82,3 +87,22 @@ def test_no_alloc_rejects_counts_above_the_fixed_payload():
     B.rlx_allreduce_tree_noalloc(x.data_ptr(), x.data_ptr(), count, count, n, B.RLX_F32,
                                  B.RLX_WIRE_NATIVE, B.RLX_SUM, None)
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("workload,nranks,count", [(4, 8, 300_000 + 77), (3, 5, 100_003)])
+def test_no_alloc_matches_oracle_twice(workload, nranks, count):
+    """Two calls in a row on two seeded inputs (first the workload's own
+    recipe and seeds, then the Student-t recipe of workload 5): every element
+    of every rank equals the oracle's FP8 DDA-tree."""
+    for call, wl in enumerate((workload, 5)):
+        x = synth.rank_buffers(wl, count=count, nranks=nranks,
+                               dtype=synth.WORKLOADS[workload].dtype)
+        xt = torch.from_numpy(x.view(np.int16) if x.dtype == np.uint16 else x).cuda()
+        out = torch.zeros_like(xt)
+        d = B.RLX_BF16 if x.dtype == np.uint16 else B.RLX_F32
+        B.rlx_allreduce_tree_noalloc(xt.data_ptr(), out.data_ptr(), count, count, nranks, d,
+                                     B.RLX_WIRE_FP8_E4M3, B.RLX_SUM, None)
+        torch.cuda.synchronize()
+        got = out.cpu().numpy().view(x.dtype)
+        ref = oracle.allreduce_tree(x, wire=oracle.FP8)
+        assert np.array_equal(got.view(np.uint8), ref.view(np.uint8)), "call %d differs" % call
