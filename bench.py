@@ -6,8 +6,8 @@ simulated ranks x 16,777,216 fp32 elements (64 MiB per rank, N(0,1) with 1%
 of the elements scaled x100 as outliers -- the >= 16 MB low-precision message
 size the RCCLX pages target):
 
-    quantise, dequantise (128-block FP8 E4M3),
-    DDA-flat allreduce    (native fp32 wire, FP8 wire),
+    quantise (128-block FP8 E4M3), DDA-flat allreduce (native fp32 wire),
+    dequantise, DDA-flat allreduce (FP8 wire),
     DDA-tree allreduce    (native fp32 wire, FP8 wire: fused
                            dequantise-sum-requantise pass + all-gather pass),
     reduce-scatter, all-gather, alltoall (native and FP8 wire).
@@ -16,7 +16,13 @@ size the RCCLX pages target):
 bytes of all operations (inputs read once, outputs written once, plus the
 tree's wire payload written by pass 1 and read by pass 2) divided by the
 device time of the timed steps.  Every operation touches >= 576 MiB, far more
-than the 126 MB L2, so no flush is needed between steps.
+than the 126 MB L2, so no flush is needed between steps; dequantise runs after
+the 1 GiB DDA-flat pass, not straight after quantise, so it reads the codes
+from HBM.  `roofline` is the slowest single-kernel operation against the
+measured copy bandwidth, and `roofline.target` the FP8 DDA-tree allreduce
+(the fused low-precision allreduce the >= 16 MB target is quoted on).
+`e2e` is that one collective end to end: each step uploads the 512 MiB
+input from pinned host memory, runs it and downloads the 512 MiB result.
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference]
 
@@ -76,6 +82,8 @@ def op_bytes(count: int, nranks: int, esize: int = 4) -> dict[str, int]:
 
 
 OPS = list(op_bytes(COUNT, NRANKS).keys())
+# the operation the >= 16 MB low-precision target is quoted on
+TARGET_OP = "allreduce_tree_fp8"
 KERNELS_PER_OP = {op: (2 if op.startswith("allreduce_tree") else 1) for op in OPS}
 
 
@@ -236,12 +244,14 @@ class Step:
         y1, y2 = self.y1.data_ptr(), self.y2.data_ptr()
         r1, r2 = self.rs1.data_ptr(), self.rs2.data_ptr()
         F, NAT, FP8 = B.RLX_F32, B.RLX_WIRE_NATIVE, B.RLX_WIRE_FP8_E4M3
+        # dequantise runs after DDA-flat, so that the 1 GiB flat pass has
+        # pushed quantise's codes out of L2 before dequantise reads them
         return [
             ("quantize_fp8", lambda: B.rlx_quantize_fp8(x, F, n, c, p, self.codes.data_ptr(),
                                                         self.scales.data_ptr(), stream)),
+            ("allreduce_flat_native", lambda: B.rlx_allreduce_flat(x, o1, c, p, n, F, NAT, B.RLX_SUM, stream)),
             ("dequantize_fp8", lambda: B.rlx_dequantize_fp8(self.codes.data_ptr(), self.scales.data_ptr(),
                                                             n, c, p, y2, F, stream)),
-            ("allreduce_flat_native", lambda: B.rlx_allreduce_flat(x, o1, c, p, n, F, NAT, B.RLX_SUM, stream)),
             ("allreduce_flat_fp8", lambda: B.rlx_allreduce_flat(x, o2, c, p, n, F, FP8, B.RLX_SUM, stream)),
             ("allreduce_tree_native", lambda: B.rlx_allreduce_tree(x, o1, c, p, n, F, NAT, B.RLX_SUM,
                                                                    None, 0, stream)),
@@ -254,6 +264,62 @@ class Step:
             ("alltoall_native", lambda: B.rlx_alltoall(x, p, y1, p, m, n, F, NAT, stream)),
             ("alltoall_fp8", lambda: B.rlx_alltoall(x, p, y2, p, m, n, F, FP8, stream)),
         ]
+
+
+class E2ETreeFp8:
+    """End to end through the C ABI, one collective per step: copy the rank
+    buffers from pinned host memory to the device, run the FP8 DDA-tree
+    allreduce (fused dequantise-sum-requantise pass + all-gather pass) and
+    copy the result back to pinned host memory.  Uploads, kernels and
+    downloads run on three streams with two device batches, so step k's
+    upload and step k-1's download overlap step k's kernels.  Calling the
+    object with a step count returns the device time of those steps (ms),
+    from the first upload's start to the last download's end."""
+
+    def __init__(self, x_host: np.ndarray, dev):
+        import torch
+        from precision_collective_reduction_fp32_b200 import binding as B
+        self.B, self.torch = B, torch
+        self.n, self.c = x_host.shape
+        self.wsb = B.rlx_workspace_bytes(B.RLX_COLL_ALLREDUCE_TREE, self.c, self.n, B.RLX_F32,
+                                         B.RLX_WIRE_FP8_E4M3)
+        self.host_in = torch.from_numpy(x_host).pin_memory()
+        self.host_out = [torch.empty((self.n, self.c), dtype=torch.float32).pin_memory()
+                         for _ in range(2)]
+        self.dx = [torch.empty((self.n, self.c), dtype=torch.float32, device=dev) for _ in range(2)]
+        self.dy = [torch.empty_like(self.dx[0]) for _ in range(2)]
+        self.ws = [torch.empty(self.wsb, dtype=torch.uint8, device=dev) for _ in range(2)]
+        self.stream = torch.cuda.current_stream(dev)
+        self.s_in, self.s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        self.h2d_bytes = self.d2h_bytes = self.n * self.c * 4
+
+    def __call__(self, nsteps: int) -> float:
+        torch, B = self.torch, self.B
+        n, c, sp = self.n, self.c, self.stream.cuda_stream or None
+        ev = lambda: torch.cuda.Event(enable_timing=True)
+        start = ev()
+        ev_in, ev_c, ev_out = ([ev() for _ in range(nsteps)] for _ in range(3))
+        start.record(self.s_in)
+        for k in range(nsteps):
+            b = k % 2
+            with torch.cuda.stream(self.s_in):
+                if k >= 2:
+                    self.s_in.wait_event(ev_c[k - 2])      # batch b's input is free again
+                self.dx[b].copy_(self.host_in, non_blocking=True)
+                ev_in[k].record(self.s_in)
+            self.stream.wait_event(ev_in[k])
+            if k >= 2:
+                self.stream.wait_event(ev_out[k - 2])      # batch b's result was read out
+            B.rlx_allreduce_tree(self.dx[b].data_ptr(), self.dy[b].data_ptr(), c, c, n, B.RLX_F32,
+                                 B.RLX_WIRE_FP8_E4M3, B.RLX_SUM, self.ws[b].data_ptr(), self.wsb,
+                                 sp)
+            ev_c[k].record(self.stream)
+            with torch.cuda.stream(self.s_out):
+                self.s_out.wait_event(ev_c[k])
+                self.host_out[b].copy_(self.dy[b], non_blocking=True)
+                ev_out[k].record(self.s_out)
+        torch.cuda.synchronize()
+        return start.elapsed_time(ev_out[-1])
 
 
 def run_gpu(args, rank: int, world: int) -> dict | None:
@@ -327,48 +393,19 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
             per_op_ms[name] += ev[k][i].elapsed_time(ev[k][i + 1])
     per_op_total_ms = ev[0][0].elapsed_time(ev[K - 1][-1])
 
-    # ---- end to end: every step copies its inputs from pinned host memory
-    # and its result (the FP8 tree allreduce output) back to pinned host
-    # memory.  Copies run on their own streams, so step k's upload and step
-    # k-1's download overlap step k's kernels; two device batches alternate.
+    # ---- end to end, one collective (the FP8 DDA-tree allreduce, the
+    # operation the >= 16 MB target is quoted on): upload, kernels, download
     Ke = max(1, min(K, args.e2e_steps))
-    host_in = torch.from_numpy(x_host).pin_memory()
-    host_out = [torch.empty((NRANKS, count), dtype=torch.float32).pin_memory() for _ in range(2)]
-    batches = [step, Step(x_host, dev)]
-    batch_ops = [b.ops(sp) for b in batches]
-    if args.only:
-        batch_ops = [[(n, f) for n, f in bo if n in dict(ops)] for bo in batch_ops]
-    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-
-    def e2e(nsteps):
-        ev = lambda: torch.cuda.Event(enable_timing=True)
-        start, ev_in, ev_c, ev_out = ev(), [ev() for _ in range(nsteps)], \
-            [ev() for _ in range(nsteps)], [ev() for _ in range(nsteps)]
-        start.record(s_in)
-        for k in range(nsteps):
-            b = k % 2
-            with torch.cuda.stream(s_in):
-                if k >= 2:
-                    s_in.wait_event(ev_c[k - 2])      # batch b's inputs are free again
-                batches[b].x[:, :count].copy_(host_in, non_blocking=True)
-                ev_in[k].record(s_in)
-            stream.wait_event(ev_in[k])
-            if k >= 2:
-                stream.wait_event(ev_out[k - 2])      # batch b's result was read out
-            for _, f in batch_ops[b]:
-                f()
-            ev_c[k].record(stream)
-            with torch.cuda.stream(s_out):
-                s_out.wait_event(ev_c[k])
-                host_out[b].copy_(batches[b].out[:, :count], non_blocking=True)
-                ev_out[k].record(s_out)
-        torch.cuda.synchronize()
-        return start.elapsed_time(ev_out[-1])
-
-    e2e(2)
+    if world > 1:
+        # the step's buffers are no longer needed: make room on the device
+        del ops, step
+        torch.cuda.empty_cache()
+    e2e_run = E2ETreeFp8(x_host, dev)
+    e2e_run(2)
     barrier()
-    e2e_ms = max_over_ranks(e2e(Ke), dev)
+    e2e_ms = max_over_ranks(e2e_run(Ke), dev)
     barrier()
+    del e2e_run
     if rank != 0:
         return None
 
@@ -380,11 +417,17 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         gbs = bytes_[name] / (ms * 1e-3) / 1e9
         per_op[name] = {"us": round(ms * 1e3, 2), "GB/s": round(gbs, 1),
                         "Gelem/s": round(NRANKS * count / (ms * 1e-3) / 1e9, 1),
-                        "frac": round(gbs / peak, 3), "MiB": round(bytes_[name] / MIB, 1)}
+                        "frac": round(gbs / peak, 3),
+                        "frac_nominal": round(gbs / HBM_NOMINAL_GBS, 3),
+                        "MiB": round(bytes_[name] / MIB, 1)}
     single = [n for n in per_op_ms if KERNELS_PER_OP[n] == 1]
     dom = max(single, key=lambda n: per_op_ms[n])
     dom_gbs = per_op[dom]["GB/s"]
     traffic = recorded_traffic(dom)
+    peak_desc = ("%s HBM copy bandwidth (read + write bytes of a 1 GiB device copy); read-heavy "
+                 "operations can exceed it, so every fraction is also given against the nominal "
+                 "%.0f GB/s" % (peak_kind, HBM_NOMINAL_GBS))
+    e2e_bytes = op_bytes(count, NRANKS)[TARGET_OP]
     res = {
         "metric": "emulated N=8 allreduce effective HBM GB/s (fp32 & FP8) and % of B200 HBM peak",
         "value": round(value, 1),
@@ -401,33 +444,47 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
         "data": "synthetic",
         "config": {
             "workload": "N=8 simulated ranks x fp32[16,777,216] (64 MiB/rank), N(0,1) with 1% "
-                        "x100 outliers; one step = quantise, dequantise, DDA-flat and DDA-tree "
-                        "allreduce (native and FP8 wire), reduce-scatter, all-gather, alltoall "
-                        "(native and FP8 wire)",
+                        "x100 outliers; one step = quantise, DDA-flat native, dequantise, DDA-flat "
+                        "FP8, DDA-tree allreduce (native and FP8 wire), reduce-scatter, all-gather, "
+                        "alltoall (native and FP8 wire)",
             "nranks": NRANKS, "count": count, "elem": "fp32", "fp8": "e4m3, 128-block fp32 scales",
             "bytes_per_step": step_bytes,
-            "l2": "no flush: every operation streams >= 576 MiB, > 126 MB L2",
+            "l2": "no flush: every operation streams >= 576 MiB, > 126 MB L2; dequantise "
+                  "follows the 1 GiB DDA-flat pass, not quantise",
             "parallelism": "independent batch per GPU" if world > 1 else "single GPU",
         },
         "hbm_frac": round(value / world / peak, 3),
         "hbm_frac_nominal": round(value / world / HBM_NOMINAL_GBS, 3),
+        "peak_note": peak_desc,
         "ops": per_op,
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": dom_gbs, "peak": peak,
                      "unit": "GB/s", "frac": round(dom_gbs / peak, 3), "traffic": traffic,
-                     "algorithmic_bytes": bytes_[dom], "peak_kind": peak_kind},
+                     "algorithmic_bytes": bytes_[dom], "peak_kind": peak_kind + " copy"},
         "gpu_launches": K * sum(KERNELS_PER_OP[n] for n in bytes_),
         "gpu_launches_breakdown_pass": K * sum(KERNELS_PER_OP[n] for n in bytes_),
-        "gpu_launches_e2e": Ke * sum(KERNELS_PER_OP[n] for n in bytes_),
+        "gpu_launches_e2e": Ke * KERNELS_PER_OP[TARGET_OP],
         "clocks": clk,
-        "e2e": {"value": round(whole_job_gbs(world, step_bytes, Ke, e2e_ms), 1), "unit": "GB/s",
+        "e2e": {"value": round(whole_job_gbs(world, e2e_bytes, Ke, e2e_ms), 1), "unit": "GB/s",
                 "h2d_bytes_per_step": NRANKS * count * 4, "d2h_bytes_per_step": NRANKS * count * 4,
                 "ms_per_step": round(e2e_ms / Ke, 3), "steps": Ke,
+                "operation": TARGET_OP,
+                "numerator": "the operation's algorithmic HBM bytes (%d per step)" % e2e_bytes,
+                "pcie_GBs": round(world * 2 * NRANKS * count * 4 * Ke / (e2e_ms * 1e-3) / 1e9, 1),
                 "overlap": "uploads, kernels and downloads on three streams, two device batches"},
     }
+    if TARGET_OP in per_op:
+        t = per_op[TARGET_OP]
+        res["roofline"]["target"] = {
+            "operation": TARGET_OP, "kernels": KERNELS_PER_OP[TARGET_OP],
+            "workload": "N=8 x fp32[16,777,216] (64 MiB per rank)",
+            "us": t["us"], "achieved": t["GB/s"], "peak": peak, "unit": "GB/s",
+            "frac": t["frac"], "frac_nominal": t["frac_nominal"],
+            "algorithmic_bytes": bytes_[TARGET_OP], "traffic": recorded_traffic(TARGET_OP),
+            "goal": ">= 0.70 of the HBM roofline for the fused FP8 allreduce on >= 16 MB messages"}
     if world == 1 and not args.only and not args.no_latency:
         res["small_messages"] = small_message_latency(dev)
     if world == 1 and not args.only and not args.no_workloads:
-        del ops, batch_ops, batches, step
+        del ops, step
         torch.cuda.empty_cache()
         res["workloads"] = workload_suite(dev, peak)
     if count != COUNT or args.only:
@@ -639,6 +696,85 @@ def workload_suite(dev, peak: float, reps: int = 20, scale: int = 1) -> dict:
     return res
 
 
+# ------------------------------------------------- quotient ablation
+
+def quotient_ablation(dev, reps: int = 20) -> dict:
+    """Profiling mode: what the correctly rounded quotient costs.  Times the
+    FP8-wire operations with the product build (quotient fl32(x / s) by
+    Markstein corrections) and with two profiling builds of the same sources
+    (build.VARIANTS: x * fl32(448 / amax), and CUDA's IEEE division for every
+    element), on workload 4 (N=8 x fp32[16,777,216]) and on the bf16 prefill
+    buffers (N=8 x bf16[33,554,432]), inputs drawn on the device; and counts
+    the quantised codes and DDA-tree results in which each variant differs
+    from the product build."""
+    import torch
+    from precision_collective_reduction_fp32_b200 import binding as B
+    from precision_collective_reduction_fp32_b200 import build as rlx_build
+    from precision_collective_reduction_fp32_b200 import synth
+    libs = {"correctly_rounded (product)": B.lib()}
+    for name in rlx_build.VARIANTS:
+        libs[name] = B.load(rlx_build.build_variant(name))
+    st = torch.cuda.current_stream(dev)
+    sp = st.cuda_stream or None
+    FP8, SUM = B.RLX_WIRE_FP8_E4M3, B.RLX_SUM
+
+    def ok(rc):
+        if rc != B.RLX_OK:
+            raise RuntimeError("rlx call failed: %d" % rc)
+
+    res = {"us": {}, "differs_from_product": {}}
+    for wl, dcode, esize, tag in ((4, B.RLX_F32, 4, "lp_allreduce_fp32_8x16777216"),
+                                  (3, B.RLX_BF16, 2, "prefill_bf16_8x33554432")):
+        x = synth.device_rank_buffers(wl, dev)
+        n, c = x.shape
+        m = c // n
+        y = torch.empty_like(x)
+        rs = torch.empty((n, m), dtype=x.dtype, device=dev)
+        codes = torch.empty((n, c), dtype=torch.uint8, device=dev)
+        scales = torch.empty((n, c // BLOCK), dtype=torch.float32, device=dev)
+        wsb = B.rlx_workspace_bytes(B.RLX_COLL_ALLREDUCE_TREE, c, n, dcode, FP8)
+        ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+        ob = op_bytes(c, n, esize)
+        ref_codes = ref_tree = None
+        for lname, L in libs.items():
+            calls = {
+                "quantize_fp8": lambda: ok(L.rlx_quantize_fp8(x.data_ptr(), dcode, n, c, c,
+                                                              codes.data_ptr(), scales.data_ptr(), sp)),
+                "allreduce_flat_fp8": lambda: ok(L.rlx_allreduce_flat(x.data_ptr(), y.data_ptr(), c, c,
+                                                                      n, dcode, FP8, SUM, sp)),
+                "allreduce_tree_fp8": lambda: ok(L.rlx_allreduce_tree(x.data_ptr(), y.data_ptr(), c, c,
+                                                                      n, dcode, FP8, SUM, ws.data_ptr(),
+                                                                      wsb, sp)),
+                "reduce_scatter_fp8": lambda: ok(L.rlx_reduce_scatter(x.data_ptr(), c, rs.data_ptr(), m,
+                                                                      m, n, dcode, FP8, SUM, sp)),
+                "all_gather_fp8": lambda: ok(L.rlx_all_gather(rs.data_ptr(), m, y.data_ptr(), c, m, n,
+                                                              dcode, FP8, sp)),
+                "alltoall_fp8": lambda: ok(L.rlx_alltoall(x.data_ptr(), c, y.data_ptr(), c, m, n,
+                                                          dcode, FP8, sp)),
+            }
+            row = {}
+            for op, f in calls.items():
+                us = _timed_us(f, st, reps)
+                row[op] = {"us": round(us, 2), "GB/s": round(ob[op] / (us * 1e-6) / 1e9, 1)}
+            row["fp8_ops_total_us"] = round(sum(v["us"] for v in row.values()), 1)
+            res["us"].setdefault(lname, {})[tag] = row
+            calls["quantize_fp8"]()
+            calls["allreduce_tree_fp8"]()
+            torch.cuda.synchronize()
+            if ref_codes is None:
+                ref_codes, ref_tree = codes.clone(), y.clone()
+            else:
+                it = torch.int16 if x.dtype == torch.bfloat16 else torch.int32
+                res["differs_from_product"].setdefault(lname, {})[tag] = {
+                    "quantize_codes": int((codes != ref_codes).sum().item()),
+                    "codes_total": codes.numel(),
+                    "tree_fp8_elements": int((y.view(it) != ref_tree.view(it)).sum().item()),
+                    "elements_total": y.numel()}
+        del x, y, rs, codes, scales, ws, ref_codes, ref_tree
+        torch.cuda.empty_cache()
+    return res
+
+
 # --------------------------------------------------------------- CPU oracle
 
 def oracle_step(xs: np.ndarray) -> None:
@@ -724,6 +860,10 @@ def main(argv=None):
                          "(--steps calls each)")
     ap.add_argument("--suite-scale", type=int, default=1,
                     help="profiling: divide the other workloads' counts by this")
+    ap.add_argument("--quotient-ablation", action="store_true",
+                    help="profiling: time the FP8 operations with the correctly rounded "
+                         "quotient against two profiling builds (reciprocal multiply, IEEE "
+                         "division for every element); --steps calls each")
     ap.add_argument("--count", type=int, default=COUNT,
                     help="elements per rank (profiling cases only; the benchmark is 16,777,216)")
     ap.add_argument("--only", default="",
@@ -740,6 +880,14 @@ def main(argv=None):
         print(json.dumps({"workloads": workload_suite(torch.device("cuda", 0), peaks()[0],
                                                       reps=args.steps, scale=args.suite_scale),
                           "note": "PROFILING CASE, counts / %d" % args.suite_scale}), flush=True)
+        return 0
+    if args.quotient_ablation:
+        import torch
+        torch.cuda.set_device(0)
+        print(json.dumps({"quotient_ablation": quotient_ablation(torch.device("cuda", 0),
+                                                                 reps=args.steps),
+                          "note": "PROFILING CASE: product build against profiling builds"}),
+              flush=True)
         return 0
     if args.impl == "reference":
         res = run_reference(args, rank)
