@@ -518,16 +518,23 @@ def small_message_latency(dev, reps: int = 200, graph_reps: int = 50) -> dict:
         ws = torch.empty(max(B.rlx_workspace_bytes(B.RLX_COLL_ALLREDUCE_TREE, c, n, dcode,
                                                    B.RLX_WIRE_FP8_E4M3), 16),
                          dtype=torch.uint8, device=dev)
+        # the one-launch tree: zeroed synchronisation words (each call leaves them zero)
+        fws = torch.zeros(B.rlx_workspace_bytes(B.RLX_COLL_ALLREDUCE_TREE_FUSED, c, n, dcode,
+                                                B.RLX_WIRE_FP8_E4M3), dtype=torch.uint8, device=dev)
         row = {}
-        for algo in ("flat", "tree"):
+        for algo in ("flat", "tree", "tree_fused"):
             for wname, wire in (("native", B.RLX_WIRE_NATIVE), ("fp8", B.RLX_WIRE_FP8_E4M3)):
                 def call(stream_ptr):
                     if algo == "flat":
                         B.rlx_allreduce_flat(x.data_ptr(), out.data_ptr(), c, c, n, dcode, wire,
                                              B.RLX_SUM, stream_ptr)
-                    else:
+                    elif algo == "tree":
                         B.rlx_allreduce_tree(x.data_ptr(), out.data_ptr(), c, c, n, dcode, wire,
                                              B.RLX_SUM, ws.data_ptr(), ws.numel(), stream_ptr)
+                    else:
+                        B.rlx_allreduce_tree_fused(x.data_ptr(), out.data_ptr(), c, c, n, dcode,
+                                                   wire, B.RLX_SUM, fws.data_ptr(), fws.numel(),
+                                                   None, 0, stream_ptr)
                 st = torch.cuda.current_stream(dev)
                 for _ in range(20):
                     call(st.cuda_stream or None)
@@ -631,21 +638,28 @@ def workload_suite(dev, peak: float, reps: int = 20, scale: int = 1) -> dict:
         out = torch.empty_like(x)
         ws = torch.empty(max(B.rlx_workspace_bytes(B.RLX_COLL_ALLREDUCE_TREE, c, n, dcode, FP8), 16),
                          dtype=torch.uint8, device=dev)
+        fws = torch.zeros(B.rlx_workspace_bytes(B.RLX_COLL_ALLREDUCE_TREE_FUSED, c, n, dcode, FP8),
+                          dtype=torch.uint8, device=dev)
         ob = op_bytes(c, n, esize)
         row = {}
-        for algo in ("flat", "tree"):
+        for algo in ("flat", "tree", "tree_fused"):
             for wname, wire in wires:
                 if algo == "flat":
                     f = lambda w=wire: B.rlx_allreduce_flat(x.data_ptr(), out.data_ptr(), c, c, n,
                                                             dcode, w, SUM, sp)
-                else:
+                elif algo == "tree":
                     f = lambda w=wire: B.rlx_allreduce_tree(x.data_ptr(), out.data_ptr(), c, c, n,
                                                             dcode, w, SUM, ws.data_ptr(),
                                                             ws.numel(), sp)
-                nb = ob["allreduce_%s_%s" % (algo, wname)]
+                else:
+                    f = lambda w=wire: B.rlx_allreduce_tree_fused(x.data_ptr(), out.data_ptr(), c, c,
+                                                                  n, dcode, w, SUM, fws.data_ptr(),
+                                                                  fws.numel(), None, 0, sp)
+                # the one-launch tree moves the same algorithmic bytes as the tree
+                nb = ob["allreduce_%s_%s" % ("tree" if algo == "tree_fused" else algo, wname)]
                 us = _cold_us(f, st, cold, reps, dirty) if cold is not None else _timed_us(f, st, reps)
                 row["allreduce_%s_%s" % (algo, wname)] = entry(us, nb)
-        del out, ws
+        del out, ws, fws
         return row
 
     def chunked(x, dcode, esize, quantise):

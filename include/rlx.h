@@ -85,7 +85,8 @@ typedef enum {
     RLX_ERR_UNSUPPORTED = 3,  /* reduction op other than SUM                      */
     RLX_ERR_WORKSPACE = 4,    /* workspace missing, too small or misaligned       */
     RLX_ERR_CUDA = 5,         /* a CUDA call failed (see rlx_last_cuda_error)     */
-    RLX_ERR_TIMEOUT = 6       /* reserved for bounded device-side waits           */
+    RLX_ERR_TIMEOUT = 6       /* a bounded device-side wait ran out (written to a
+                                 call's status word, see rlx_allreduce_tree_fused) */
 } rlx_status;
 
 typedef enum { RLX_F32 = 0, RLX_BF16 = 1 } rlx_dtype;
@@ -96,7 +97,8 @@ typedef enum {
     RLX_COLL_ALLREDUCE_TREE = 1,
     RLX_COLL_REDUCE_SCATTER = 2,
     RLX_COLL_ALL_GATHER = 3,
-    RLX_COLL_ALLTOALL = 4
+    RLX_COLL_ALLTOALL = 4,
+    RLX_COLL_ALLREDUCE_TREE_FUSED = 5
 } rlx_coll;
 
 /*
@@ -148,6 +150,51 @@ RLX_API rlx_status rlx_allreduce_flat(const void *send, void *recv, size_t count
 RLX_API rlx_status rlx_allreduce_tree(const void *send, void *recv, size_t count, size_t stride,
                               int nranks, rlx_dtype dtype, rlx_wire wire, rlx_op op,
                               void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * DDA-tree SUM allreduce in ONE kernel launch: the same results as
+ * rlx_allreduce_tree, bit for bit, but the all-gather of chunk c starts as
+ * soon as chunk c is reduced instead of after the whole reduce-scatter pass,
+ * and there is no second launch (the pages credit the DDA-tree with
+ * near-constant latency: "Meta open-sources RCCLX", infolabhq pt, section
+ * "Direct Data Access (DDA) — De O(N) para O(1) de Latência").  Meant for
+ * small and medium messages, where launch latency dominates.
+ *
+ * The kernel's CTAs coordinate through the workspace: the reduce-scatter
+ * work of chunk c adds to a per-chunk count with release semantics, and the
+ * all-gather work of chunk c waits, with acquire loads, until that count is
+ * complete.  Every wait is bounded: it gives up after wait_limit_ns
+ * nanoseconds of the GPU's global timer (0 = RLX_DEFAULT_WAIT_NS), or after a
+ * fixed number of polls if the timer does not advance; the kernel then skips
+ * the work that depended on the wait, returns, and reports RLX_ERR_TIMEOUT in
+ * *status.  No wait can block forever on work that is never started: work is
+ * handed out in order, all of the reduce-scatter work before any of the
+ * all-gather work, and only to CTAs that are already running.
+ *
+ * workspace: device memory of at least
+ *   rlx_workspace_bytes(RLX_COLL_ALLREDUCE_TREE_FUSED, count, nranks, dtype, wire)
+ * bytes, 16-byte aligned, not overlapping send/recv.  Its first
+ * RLX_TREE_SYNC_BYTES bytes are synchronisation words that must be ZERO
+ * before the first call on a workspace (cudaMemset it once); every call
+ * leaves them zero when its kernel ends, after a timeout too.  Word 4 + c
+ * (32-bit) counts the reduce-scatter work finished on chunk c; chunk c is
+ * ready when that count, read as a signed number, reaches the chunk's total
+ * (so a count preset to INT_MIN never gets there).  The rest
+ * (FP8 wire only) carries the reduced chunks' FP8 payload.  Calls that can
+ * run at the same time need a workspace each.
+ * status: NULL, or a device int the kernel sets to RLX_OK or RLX_ERR_TIMEOUT
+ *   when it ends (read it after synchronising).  On RLX_ERR_TIMEOUT recv is
+ *   unspecified.
+ * The host return value covers argument checks and the launch only.
+ * Everything else as rlx_allreduce_tree (in place allowed).
+ */
+#define RLX_TREE_SYNC_BYTES 256
+#define RLX_DEFAULT_WAIT_NS 1000000000ull
+RLX_API rlx_status rlx_allreduce_tree_fused(const void *send, void *recv, size_t count,
+                                            size_t stride, int nranks, rlx_dtype dtype,
+                                            rlx_wire wire, rlx_op op, void *workspace,
+                                            size_t workspace_bytes, int *status,
+                                            uint64_t wait_limit_ns, void *stream);
 
 /*
  * ReduceScatter: send [nranks][send_stride >= nranks*m], recv

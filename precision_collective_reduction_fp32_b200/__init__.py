@@ -19,16 +19,18 @@ import torch
 
 from . import binding as _b
 from .binding import (RLX_BF16, RLX_BLOCK, RLX_COLL_ALL_GATHER, RLX_COLL_ALLREDUCE_FLAT,
-                      RLX_COLL_ALLREDUCE_TREE, RLX_COLL_ALLTOALL, RLX_COLL_REDUCE_SCATTER,
-                      RLX_F32, RLX_MAX_RANKS, RLX_SUM, RLX_WIRE_FP8_E4M3, RLX_WIRE_NATIVE,
-                      RlxError, rlx_all_gather, rlx_allreduce_flat, rlx_allreduce_tree,
+                      RLX_COLL_ALLREDUCE_TREE, RLX_COLL_ALLREDUCE_TREE_FUSED, RLX_COLL_ALLTOALL,
+                      RLX_COLL_REDUCE_SCATTER, RLX_ERR_TIMEOUT, RLX_F32, RLX_MAX_RANKS, RLX_OK,
+                      RLX_SUM, RLX_WIRE_FP8_E4M3, RLX_WIRE_NATIVE, RlxError, rlx_all_gather,
+                      rlx_allreduce_flat, rlx_allreduce_tree, rlx_allreduce_tree_fused,
                       rlx_allreduce_tree_noalloc, rlx_alltoall, rlx_dequantize_fp8,
                       rlx_quantize_fp8, rlx_reduce_scatter, rlx_status_string,
                       rlx_workspace_bytes)
 
 __all__ = ["allreduce", "reduce_scatter", "all_gather", "alltoall", "quantize_fp8",
            "dequantize_fp8", "workspace_bytes", "RlxError", "rlx_allreduce_flat",
-           "rlx_allreduce_tree", "rlx_allreduce_tree_noalloc", "rlx_reduce_scatter",
+           "rlx_allreduce_tree", "rlx_allreduce_tree_noalloc", "rlx_allreduce_tree_fused",
+           "rlx_reduce_scatter",
            "rlx_all_gather", "rlx_alltoall", "rlx_quantize_fp8", "rlx_dequantize_fp8",
            "rlx_workspace_bytes", "rlx_status_string", "default_wire"]
 
@@ -96,14 +98,31 @@ def workspace_bytes(coll: int, count: int, nranks: int, dtype: torch.dtype,
     return rlx_workspace_bytes(coll, count, nranks, d, _wire(wire))
 
 
+def fused_tree_workspace(x: torch.Tensor, wire: str | None = None) -> torch.Tensor:
+    """A zeroed workspace for algo="tree_fused" on rank buffers shaped like x
+    (reusable by later calls on the same stream: each call leaves its
+    synchronisation words zero)."""
+    n, count, _ = _rows(x)
+    need = rlx_workspace_bytes(RLX_COLL_ALLREDUCE_TREE_FUSED, count, n, _dtype(x), _wire(wire))
+    return torch.zeros(max(need, 16), dtype=torch.uint8, device=x.device)
+
+
 def allreduce(x: torch.Tensor, algo: str = "flat", wire: str | None = None,
-              out: torch.Tensor | None = None, workspace: torch.Tensor | None = None):
-    """SUM allreduce over the ranks (rows) of x.  out may be x (in place)."""
+              out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+              status: torch.Tensor | None = None, wait_limit_ns: int = 0):
+    """SUM allreduce over the ranks (rows) of x.  out may be x (in place).
+
+    algo: "flat" (DDA-flat), "tree" (DDA-tree, two launches) or "tree_fused"
+    (DDA-tree in one launch with bounded chunk-ready waits; its workspace
+    must start zeroed, see fused_tree_workspace, and `status`, an int32 CUDA
+    tensor of one element, receives RLX_OK or RLX_ERR_TIMEOUT)."""
     n, count, stride = _rows(x)
     out = torch.empty_like(x) if out is None else out
     if out.shape != x.shape or out.dtype != x.dtype or _rows(out)[2] != stride:
         raise ValueError("out must match x in shape, dtype and row stride")
     d, w = _dtype(x), _wire(wire)
+    if status is not None and algo != "tree_fused":
+        raise ValueError("status applies to algo='tree_fused' only")
     if algo == "flat":
         rlx_allreduce_flat(x.data_ptr(), out.data_ptr(), count, stride, n, d, w, RLX_SUM, _stream())
     elif algo == "tree":
@@ -114,8 +133,17 @@ def allreduce(x: torch.Tensor, algo: str = "flat", wire: str | None = None,
         wb = workspace.numel() * workspace.element_size() if workspace is not None else 0
         rlx_allreduce_tree(x.data_ptr(), out.data_ptr(), count, stride, n, d, w, RLX_SUM, wp, wb,
                            _stream())
+    elif algo == "tree_fused":
+        if workspace is None:
+            workspace = fused_tree_workspace(x, wire)
+        if status is not None and (status.dtype != torch.int32 or not status.is_cuda):
+            raise ValueError("status must be an int32 CUDA tensor")
+        rlx_allreduce_tree_fused(x.data_ptr(), out.data_ptr(), count, stride, n, d, w, RLX_SUM,
+                                 workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                 status.data_ptr() if status is not None else None, wait_limit_ns,
+                                 _stream())
     else:
-        raise ValueError("algo must be 'flat' or 'tree'")
+        raise ValueError("algo must be 'flat', 'tree' or 'tree_fused'")
     return out
 
 

@@ -38,42 +38,61 @@ def _deps() -> list[str]:
                                   if f.endswith((".cuh", ".h"))]
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+def stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(p) > t for p in _deps())
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    if not force and not stale():
-        return LIB
-    os.makedirs(OBJ, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None,
+          lib: str = LIB, obj: str = OBJ) -> str:
+    if not force and not stale(lib):
+        return lib
+    os.makedirs(obj, exist_ok=True)
     flags = FLAGS + list(extra or [])
 
     def compile_one(src: str) -> str:
-        obj = os.path.join(OBJ, os.path.basename(src)[:-3] + ".o")
-        cmd = [NVCC, *flags, "-c", src, "-o", obj]
+        o = os.path.join(obj, os.path.basename(src)[:-3] + ".o")
+        cmd = [NVCC, *flags, "-c", src, "-o", o]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError("nvcc failed for %s:\n%s%s" % (src, r.stdout, r.stderr))
         if verbose and (r.stdout or r.stderr):
             sys.stderr.write(r.stdout + r.stderr)
-        return obj
+        return o
 
     with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
         objs = list(ex.map(compile_one, sources()))
 
-    vmap = os.path.join(OBJ, "rlx.map")
+    vmap = os.path.join(obj, "rlx.map")
     with open(vmap, "w") as f:
         f.write("{ global: rlx_*; local: *; };\n")
-    tmp = LIB + ".tmp.%d" % os.getpid()
+    os.makedirs(os.path.dirname(lib), exist_ok=True)
+    tmp = lib + ".tmp.%d" % os.getpid()
     cmd = [NVCC, *ARCH, "-shared", "-o", tmp, *objs, "-Xlinker", "--version-script=" + vmap]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("link failed:\n%s%s" % (r.stdout, r.stderr))
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
+
+
+# Profiling builds: the same sources with one compile-time switch changed,
+# written under _build/variants/<name>/ (never next to the package, so the
+# package always loads the product build).  Used by bench.py's ablation mode.
+VARIANTS = {
+    # quotient x * fl32(448 / amax) instead of the correctly rounded x / s
+    "recip_quotient": ["-DRLX_QUOTIENT=1"],
+    # CUDA's IEEE division for every element
+    "ieee_div_quotient": ["-DRLX_QUOTIENT=2"],
+}
+
+
+def build_variant(name: str, force: bool = False) -> str:
+    base = os.path.join(ROOT, "_build", "variants", name)
+    return build(force=force, extra=VARIANTS[name], lib=os.path.join(base, "librlx.so"),
+                 obj=os.path.join(base, "obj"))
 
 
 if __name__ == "__main__":

@@ -145,8 +145,10 @@ int rlx_last_cuda_error(void) { return g_last_cuda_error; }
 size_t rlx_workspace_bytes(rlx_coll coll, size_t count, int nranks, rlx_dtype dtype,
                            rlx_wire wire) {
     (void)dtype;
-    if (coll == RLX_COLL_ALLREDUCE_TREE && wire == RLX_WIRE_FP8_E4M3 && nranks > 1 && count > 0)
-        return tree_ws_bytes(count);
+    if (nranks <= 1 || count == 0) return 0;
+    if (coll == RLX_COLL_ALLREDUCE_TREE && wire == RLX_WIRE_FP8_E4M3) return tree_ws_bytes(count);
+    if (coll == RLX_COLL_ALLREDUCE_TREE_FUSED)
+        return RLX_TREE_SYNC_BYTES + (wire == RLX_WIRE_FP8_E4M3 ? tree_ws_bytes(count) : 0);
     return 0;
 }
 
@@ -253,6 +255,40 @@ rlx_status rlx_allreduce_tree(const void *send, void *recv, size_t count, size_t
     if (e != cudaSuccess) return from_cuda(e);
     return from_cuda(rlx::launch_tree_gather(recv, count, stride, nranks, chunk, dtype, wire,
                                              ws_codes, ws_scales, vec, s));
+}
+
+rlx_status rlx_allreduce_tree_fused(const void *send, void *recv, size_t count, size_t stride,
+                                    int nranks, rlx_dtype dtype, rlx_wire wire, rlx_op op,
+                                    void *workspace, size_t workspace_bytes, int *status,
+                                    uint64_t wait_limit_ns, void *stream) {
+    size_t bytes = 0;
+    rlx_status st = check_allreduce(send, recv, count, stride, nranks, dtype, wire, op, &bytes);
+    if (st != RLX_OK) return st;
+    if (status != nullptr && !aligned(status, alignof(int))) return RLX_ERR_ALIGNMENT;
+    if (status != nullptr && (overlap(status, sizeof(int), send, bytes) ||
+                              overlap(status, sizeof(int), recv, bytes)))
+        return RLX_ERR_INVALID_ARG;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t es = elem_size(dtype);
+    if (count == 0 || nranks == 1) {
+        // nothing waits: the status is RLX_OK as soon as the copy (if any) is queued
+        if (count != 0 && send != recv) {
+            const cudaError_t e = rlx::launch_copy(send, recv, count, dtype,
+                                                   vec_ok(RLX_WIRE_NATIVE, es, {send, recv}, {}), s);
+            if (e != cudaSuccess) return from_cuda(e);
+        }
+        return status != nullptr ? from_cuda(cudaMemsetAsync(status, 0, sizeof(int), s)) : RLX_OK;
+    }
+    const size_t need = rlx_workspace_bytes(RLX_COLL_ALLREDUCE_TREE_FUSED, count, nranks, dtype, wire);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return RLX_ERR_WORKSPACE;
+    if (overlap(workspace, need, send, bytes) || overlap(workspace, need, recv, bytes) ||
+        (status != nullptr && overlap(workspace, need, status, sizeof(int))))
+        return RLX_ERR_WORKSPACE;
+    const bool vec = vec_ok(wire, es, {send, recv}, {stride});
+    const uint64_t limit = wait_limit_ns != 0 ? wait_limit_ns : RLX_DEFAULT_WAIT_NS;
+    return from_cuda(rlx::launch_tree_fused(send, recv, count, stride, nranks,
+                                            tree_chunk(count, nranks), dtype, wire, workspace,
+                                            status, limit, vec, s));
 }
 
 // Shared checks of the three chunked collectives.

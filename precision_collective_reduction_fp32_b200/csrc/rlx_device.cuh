@@ -34,6 +34,12 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint16_t h) {
 __device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
     return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
+// Two fp32 -> two bf16 (each round-to-nearest-even) in one word, `lo` in the
+// low half: one packed conversion instead of two single ones.
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
 
 // Cache policy of the streaming loads and stores (inputs are read once,
 // outputs written once): RLX_LD_CS / RLX_ST_CS = 1 use the evict-first
@@ -104,12 +110,8 @@ __device__ __forceinline__ void store4(T *p, int valid, const float (&v)[4]) {
         if constexpr (sizeof(T) == 4) {
             st_stream(reinterpret_cast<float4 *>(p), make_float4(v[0], v[1], v[2], v[3]));
         } else {
-            uint2 q;
-            q.x = static_cast<uint32_t>(f32_to_bf16_bits(v[0])) |
-                  (static_cast<uint32_t>(f32_to_bf16_bits(v[1])) << 16);
-            q.y = static_cast<uint32_t>(f32_to_bf16_bits(v[2])) |
-                  (static_cast<uint32_t>(f32_to_bf16_bits(v[3])) << 16);
-            st_stream(reinterpret_cast<uint2 *>(p), q);
+            st_stream(reinterpret_cast<uint2 *>(p), make_uint2(bf16x2_bits(v[0], v[1]),
+                                                               bf16x2_bits(v[2], v[3])));
         }
     } else {
 #pragma unroll
@@ -168,17 +170,40 @@ __device__ __forceinline__ void widen4(const Raw4<uint16_t> &r, float (&v)[4]) {
     v[2] = __uint_as_float(r.w.y << 16); v[3] = __uint_as_float(r.w.y & 0xffff0000u);
 }
 
-// Bits of max |v| over the four elements (a non-negative float's bits; for
-// those the integer order is the value order).  bf16 magnitudes are compared
-// as 16-bit integers two at a time.
-__device__ __forceinline__ uint32_t absmax4_bits(const Raw4<float> &r) {
+// Amax keys: an unsigned word per lane whose integer order is the order of
+// max |v| over the lane's four elements, so that one warp max-reduction of the
+// keys finds a block's amax, and amax_of<T>(key) turns the winning key into
+// the amax.  fp32: the bits of max |v| (for non-negative floats the bit order
+// is the value order).  bf16: both 16-bit halves hold the bf16 bits of
+// max |v| (magnitudes compared as 16-bit integers two at a time), so the
+// 32-bit maximum over lanes is the maximum of the halves and the amax is the
+// high half widened exactly.
+__device__ __forceinline__ uint32_t amax_key(const Raw4<float> &r) {
     const float m = fmaxf(fmaxf(fabsf(__uint_as_float(r.w.x)), fabsf(__uint_as_float(r.w.y))),
                           fmaxf(fabsf(__uint_as_float(r.w.z)), fabsf(__uint_as_float(r.w.w))));
     return __float_as_uint(m);
 }
-__device__ __forceinline__ uint32_t absmax4_bits(const Raw4<uint16_t> &r) {
+// 1: a bf16 block's per-lane amax in bf16x2 max arithmetic (measured: one
+// ALU instruction less per 4 elements); 0: as 16-bit integers.
+#ifndef RLX_AMAX_BF16X2
+#define RLX_AMAX_BF16X2 1
+#endif
+__device__ __forceinline__ uint32_t amax_key(const Raw4<uint16_t> &r) {
+#if RLX_AMAX_BF16X2
+    // max(|a|, |b|) per half in bf16 arithmetic (sign = xor of the signs,
+    // cleared below); max is exact and keeps subnormals
+    uint32_t m;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(r.w.x), "r"(r.w.y));
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(m), "r"(__byte_perm(m, 0u, 0x1032)));
+    return m & 0x7fff7fffu;
+#else
     const uint32_t m = __vmaxu2(r.w.x & 0x7fff7fffu, r.w.y & 0x7fff7fffu);
-    return max(m & 0xffffu, m >> 16) << 16;
+    return __vmaxu2(m, __byte_perm(m, 0u, 0x1032));   // the larger half in both halves
+#endif
+}
+template <typename T> __device__ __forceinline__ float amax_of(uint32_t key) {
+    if constexpr (sizeof(T) == 4) return __uint_as_float(key);
+    else return __uint_as_float(key & 0xffff0000u);
 }
 
 // --------------------------------------------------------------- E4M3 codec
@@ -217,35 +242,106 @@ __device__ __forceinline__ float warp_amax4(const float (&v)[4]) {
     return __uint_as_float(__reduce_max_sync(kFull, __float_as_uint(m)));
 }
 
-// Scale of a block: s = fl32(amax / 448), and y = fl32(1 / s) when the fast
-// quotient may be used (s >= 2^-90), else 0.
+// How the quotient x / s of the quantiser is formed.  The product is built
+// with RLX_QUOTIENT=0: the correctly rounded quotient fl32(x / s), which the
+// definition of the codes requires.  The other two exist only for the
+// ablation that measures what exactness costs (a profiling build under
+// _build/, never the library the package loads):
+//   1  x * fl32(448 / amax), one multiply per element (the reciprocal form a
+//      faster quantiser would use; it changes some codes);
+//   2  __fdiv_rn(x, s) for every element (CUDA's IEEE division).
+#ifndef RLX_QUOTIENT
+#define RLX_QUOTIENT 0
+#endif
+constexpr int kQuotient = RLX_QUOTIENT;
+static_assert(kQuotient >= 0 && kQuotient <= 2, "RLX_QUOTIENT must be 0, 1 or 2");
+
+// Scale of a block: s = fl32(amax / 448), and ny = -fl32(1 / s) when the fast
+// quotient may be used (s >= 2^-90), else 0.  (RLX_QUOTIENT=1: ny =
+// -fl32(448 / amax); RLX_QUOTIENT=2: ny = 0, every element takes the IEEE
+// division.)  The reciprocal is kept negated because the quantiser works on
+// the negated quotient (see neg_quotient2).
 struct Scale {
-    float s, y;
+    float s, ny;
 };
 __device__ __forceinline__ Scale make_scale(float amax) {
     Scale r;
     r.s = __fdiv_rn(amax, kE4m3Max);
-    r.y = r.s >= kMinFastScale ? __frcp_rn(r.s) : 0.0f;
+    if constexpr (kQuotient == 0) r.ny = r.s >= kMinFastScale ? -__frcp_rn(r.s) : 0.0f;
+    else if constexpr (kQuotient == 1) r.ny = r.s >= kMinFastScale ? -__fdiv_rn(kE4m3Max, amax) : 0.0f;
+    else r.ny = 0.0f;
     return r;
 }
 
-// Scales of K blocks held by the warp at once (K <= 32, a power of two).
-// Lane l computes the division and the reciprocal for block l % K only; the
-// results are then broadcast, so a lane pays for one division instead of K.
-template <int K>
-__device__ __forceinline__ void make_scales(const float (&amax)[K], Scale (&sc)[K]) {
+// A block scale as the packed two-lane instructions take it: (s, s) and
+// (ny, ny) in adjacent registers.
+struct Scale2 {
+    float2 s, ny;
+};
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+__device__ __forceinline__ Scale2 pack(Scale sc) { return {f2(sc.s, sc.s), f2(sc.ny, sc.ny)}; }
+
+// Per-warp shared memory through which the lanes of a warp exchange block
+// amaxes and scales (a slot per warp of the 256-thread CTA).
+constexpr int kWarpsPerCta = 8;
+struct alignas(16) WarpScratch {
+    float4 scale[32];   // block k: (s, s, ny, ny)
+    uint32_t key[32];   // block k: its amax key
+};
+__device__ __forceinline__ WarpScratch &warp_scratch() {
+    __shared__ WarpScratch slot[kWarpsPerCta];
+    return slot[threadIdx.x >> 5];
+}
+
+// Block scales shared by a warp, in three steps for the K blocks of a unit
+// (K <= 32, a power of two):
+//   begin_keys()          before the first key of the unit is stored (the
+//                         previous unit's readers are done with the slot);
+//   put_keys(i, ...)      the warp-uniform amax keys (amax_key, after the max
+//                         reduction) of blocks i.. go into the slot, as soon
+//                         as they are known, so few are held in registers;
+//   publish_scales<T,K>() lane l computes the division and the reciprocal
+//                         for block l % K only, so a lane pays for one
+//                         division instead of K, and writes the scale to the
+//                         slot, where scale_of(k) reads it.  Returns true
+//                         when every block takes the fast quotient.
+__device__ __forceinline__ void begin_keys() { __syncwarp(); }
+__device__ __forceinline__ void put_keys(int i, uint32_t k0, uint32_t k1, uint32_t k2,
+                                         uint32_t k3) {
+    if ((threadIdx.x & 31) == 0)
+        *reinterpret_cast<uint4 *>(&warp_scratch().key[i]) = make_uint4(k0, k1, k2, k3);
+}
+__device__ __forceinline__ void put_key(int i, uint32_t k) {
+    if ((threadIdx.x & 31) == 0) warp_scratch().key[i] = k;
+}
+template <typename T, int K>
+__device__ __forceinline__ bool publish_scales() {
     static_assert(K >= 1 && K <= 32 && (K & (K - 1)) == 0, "K must be a power of two <= 32");
-    const int mine = threadIdx.x & (K - 1);
-    float a = amax[0];
+    WarpScratch &w = warp_scratch();
+    const int lane = threadIdx.x & 31;
+    __syncwarp();
+    const Scale own = make_scale(amax_of<T>(w.key[lane & (K - 1)]));
+    if (lane < K) w.scale[lane] = make_float4(own.s, own.s, own.ny, own.ny);
+    const bool fast = __all_sync(kFull, own.ny != 0.0f);
+    __syncwarp();
+    return fast;
+}
+// All three steps for keys already held in registers.
+template <typename T, int K>
+__device__ __forceinline__ bool publish_scales(const uint32_t (&key)[K]) {
+    begin_keys();
+    if constexpr (K % 4 == 0) {
 #pragma unroll
-    for (int k = 1; k < K; ++k)
-        if (mine == k) a = amax[k];
-    const Scale m = make_scale(a);
+        for (int k = 0; k < K; k += 4) put_keys(k, key[k], key[k + 1], key[k + 2], key[k + 3]);
+    } else {
 #pragma unroll
-    for (int k = 0; k < K; ++k) {
-        sc[k].s = __shfl_sync(kFull, m.s, k);
-        sc[k].y = __shfl_sync(kFull, m.y, k);
+        for (int k = 0; k < K; ++k) put_key(k, key[k]);
     }
+    return publish_scales<T, K>();
+}
+__device__ __forceinline__ Scale2 scale_of(int k) {
+    const float4 v = warp_scratch().scale[k];
+    return {f2(v.x, v.y), f2(v.z, v.w)};
 }
 
 // fl32(x / s), correctly rounded, from y = fl32(1/s) (s >= 2^-90).
@@ -277,19 +373,25 @@ __device__ __forceinline__ float quotient_rn(float x, float s, float y) {
 #define RLX_PACKED_F32X2 1
 #endif
 
-__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
-
-// quotient_rn on two values sharing (s, y): the same steps, two lanes each.
-__device__ __forceinline__ float2 quotient_rn2(float2 x, float s, float y) {
+// -fl32(x / s) for two values sharing a scale, exactly: quotient_rn carried
+// out on p = -q.  With ny = -y every step is the negation of quotient_rn's
+// (round to nearest is symmetric): p0 = x*ny = -q0; the residual
+// r' = s*p0 + x is -(s*q0 - x); and p1 = p0 + r'*ny is
+// -(q0 - (s*q0 - x)*y) = -q1.  Where quotient_rn's residual cancels exactly
+// to +0 this one does too, which leaves p = -q intact since q != 0 there;
+// x = +-0 gives p = -+0.  No operand needs a per-element negation.
+// (RLX_QUOTIENT=1: p = x * ny.)
+__device__ __forceinline__ float2 neg_quotient2(float2 x, const Scale2 &sc) {
 #if RLX_PACKED_F32X2
-    const float2 s2 = f2(s, s), y2 = f2(y, y), ny2 = f2(-y, -y), nx = f2(-x.x, -x.y);
-    float2 q = __fmul2_rn(x, y2);
-    float2 r = __ffma2_rn(s2, q, nx);   // s*q - x
-    q = __ffma2_rn(r, ny2, q);          // q - r*y
-    r = __ffma2_rn(s2, q, nx);
-    return __ffma2_rn(r, ny2, q);
+    float2 p = __fmul2_rn(x, sc.ny);
+    if constexpr (kQuotient == 1) return p;
+    float2 r = __ffma2_rn(sc.s, p, x);   // s*p + x = -(s*q - x)
+    p = __ffma2_rn(r, sc.ny, p);         // p - r*y
+    r = __ffma2_rn(sc.s, p, x);
+    return __ffma2_rn(r, sc.ny, p);
 #else
-    return f2(quotient_rn(x.x, s, y), quotient_rn(x.y, s, y));
+    if constexpr (kQuotient == 1) return f2(__fmul_rn(x.x, sc.ny.x), __fmul_rn(x.y, sc.ny.x));
+    return f2(-quotient_rn(x.x, sc.s.x, -sc.ny.x), -quotient_rn(x.y, sc.s.x, -sc.ny.x));
 #endif
 }
 
@@ -301,28 +403,34 @@ __device__ __forceinline__ float2 add2_rn(float2 a, float2 b) {
 #endif
 }
 
-// q = fl32(v/s) for 4 values of a block with scale sc; s == 0 gives signed
-// zeros, sc.y == 0 selects the IEEE division.  Fast: sc.y != 0 is known.
+// p = -fl32(v/s) for 4 values of a block with scale sc, exactly (signed
+// zeros included): s == 0 gives -(+-0), ny == 0 the IEEE division by -s.
+// Fast: ny != 0 is known.
 template <bool Fast>
-__device__ __forceinline__ void quotients4(const float (&v)[4], Scale sc, float (&q)[4]) {
-    if (Fast || sc.y != 0.0f) {
-        const float2 a = quotient_rn2(f2(v[0], v[1]), sc.s, sc.y);
-        const float2 b = quotient_rn2(f2(v[2], v[3]), sc.s, sc.y);
-        q[0] = a.x; q[1] = a.y; q[2] = b.x; q[3] = b.y;
-    } else if (sc.s == 0.0f) {
+__device__ __forceinline__ void neg_quotients4(const float (&v)[4], const Scale2 &sc,
+                                               float (&p)[4]) {
+    if ((Fast && kQuotient != 2) || sc.ny.x != 0.0f) {
+        const float2 a = neg_quotient2(f2(v[0], v[1]), sc);
+        const float2 b = neg_quotient2(f2(v[2], v[3]), sc);
+        p[0] = a.x; p[1] = a.y; p[2] = b.x; p[3] = b.y;
+    } else if (sc.s.x == 0.0f) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) q[k] = __fmul_rn(v[k], 0.0f);  // +-0 with v's sign
+        for (int k = 0; k < 4; ++k) p[k] = __fmul_rn(v[k], -0.0f);  // zero, sign opposite to v's
     } else {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) q[k] = __fdiv_rn(v[k], sc.s);
+        for (int k = 0; k < 4; ++k) p[k] = __fdiv_rn(v[k], -sc.s.x);
     }
 }
 
 // Quantise 4 values of a block with scale sc: code = e4m3_rne_sat(fl32(v/s)).
-__device__ __forceinline__ uint32_t quant4(const float (&v)[4], Scale sc) {
-    float q[4];
-    quotients4<false>(v, sc, q);
-    return e4m3x4_from_f32(q);
+// The E4M3 encoding is symmetric in the sign (round to nearest even, the
+// saturation bound and zero included), so the codes of -q are the codes of q
+// with the sign bit of every byte flipped back.
+template <bool Fast = false>
+__device__ __forceinline__ uint32_t quant4(const float (&v)[4], const Scale2 &sc) {
+    float p[4];
+    neg_quotients4<Fast>(v, sc, p);
+    return e4m3x4_from_f32(p) ^ 0x80808080u;
 }
 
 // Dequantise 4 packed codes with scale s: fl32(e4m3(code) * s).  The
@@ -333,23 +441,60 @@ __device__ __forceinline__ uint32_t quant4(const float (&v)[4], Scale sc) {
 __device__ __forceinline__ void dequant4(uint32_t codes, float s, float (&y)[4]) {
     const float2 a = e4m3x2_to_f32(codes & 0xffffu);
     const float2 b = e4m3x2_to_f32(codes >> 16);
+#if RLX_PACKED_F32X2
+    // the products are stored, never added, so the packed multiply is safe here
+    const float2 pa = __fmul2_rn(a, f2(s, s)), pb = __fmul2_rn(b, f2(s, s));
+    y[0] = pa.x; y[1] = pa.y; y[2] = pb.x; y[3] = pb.y;
+#else
     y[0] = __fmul_rn(a.x, s); y[1] = __fmul_rn(a.y, s);
     y[2] = __fmul_rn(b.x, s); y[3] = __fmul_rn(b.y, s);
+#endif
 }
 
-// dequantise(quantise(v)) of 4 values of a block, in place: the same steps
-// as dequant4(quant4(v, sc), sc.s, v), with each pair of codes going straight
-// from one conversion to the other instead of through a packed word.
+// dequantise(quantise(v)) of 4 values of a block, in place.  The codes of
+// the negated quotient are the codes of -q, whose values are exactly -w, so
+// fl32((-w) * (-s)) = fl32(w * s) is the dequantised value (the sign of a
+// zero included); each pair of codes goes straight from one conversion to
+// the other.
+// 1: the dequantising product of the wire is one packed FMA with a -0 addend
+// per pair: fl32(w*s + -0) = fl32(w*s) for every w*s (zeros included), and
+// the addend, formed at run time as (-s)*0, is not a constant the compiler
+// could drop to contract the product into the add that follows.  0: scalar
+// multiplies (never contracted).
+#ifndef RLX_DEQ_FFMA2
+#define RLX_DEQ_FFMA2 0
+#endif
 template <bool Fast>
-__device__ __forceinline__ void wire4(float (&v)[4], Scale sc) {
-    float q[4];
-    quotients4<Fast>(v, sc, q);
+__device__ __forceinline__ void wire4(float (&v)[4], const Scale2 &sc) {
+    float p[4];
+    neg_quotients4<Fast>(v, sc, p);
+    const float ns = -sc.s.x;
+#if RLX_DEQ_FFMA2 && RLX_PACKED_F32X2
+    const float nz = __fmul_rn(ns, 0.0f);   // -0: s >= 0
+    const float2 ns2 = f2(ns, ns), nz2 = f2(nz, nz);
 #pragma unroll
-    for (int p = 0; p < 2; ++p) {
-        const float2 w = e4m3x2_to_f32(e4m3x2_from_f32(q[2 * p], q[2 * p + 1]));
-        v[2 * p] = __fmul_rn(w.x, sc.s);
-        v[2 * p + 1] = __fmul_rn(w.y, sc.s);
+    for (int k = 0; k < 2; ++k) {
+        const float2 w = e4m3x2_to_f32(e4m3x2_from_f32(p[2 * k], p[2 * k + 1]));
+        const float2 y = __ffma2_rn(w, ns2, nz2);
+        v[2 * k] = y.x;
+        v[2 * k + 1] = y.y;
     }
+#else
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const float2 w = e4m3x2_to_f32(e4m3x2_from_f32(p[2 * k], p[2 * k + 1]));
+        v[2 * k] = __fmul_rn(w.x, ns);
+        v[2 * k + 1] = __fmul_rn(w.y, ns);
+    }
+#endif
+}
+
+// Calls f(std::true_type{}) when every block scale of the unit takes the fast
+// quotient, else f(std::false_type{}).
+template <typename F>
+__device__ __forceinline__ void with_fast(bool fast, F &&f) {
+    if (fast) f(std::true_type{});
+    else f(std::false_type{});
 }
 
 // What a receiver holds after K 128-blocks crossed the FP8 wire.  The warp
@@ -357,13 +502,13 @@ __device__ __forceinline__ void wire4(float (&v)[4], Scale sc) {
 // +0, which leaves its amax unchanged).  In place.
 template <int K>
 __device__ __forceinline__ void wire_fp8_blocks(float (&v)[K][4]) {
-    float amax[K];
+    uint32_t key[K];
 #pragma unroll
-    for (int k = 0; k < K; ++k) amax[k] = warp_amax4(v[k]);
-    Scale sc[K];
-    make_scales<K>(amax, sc);
+    for (int k = 0; k < K; ++k) key[k] = __float_as_uint(warp_amax4(v[k]));
+    with_fast(publish_scales<float, K>(key), [&](auto fast) {
 #pragma unroll
-    for (int k = 0; k < K; ++k) wire4<false>(v[k], sc[k]);
+        for (int k = 0; k < K; ++k) wire4<decltype(fast)::value>(v[k], scale_of(k));
+    });
 }
 
 // ----------------------------------------------------------- work layout
@@ -454,14 +599,6 @@ template <int NR, bool EXACT, typename F>
 __device__ __forceinline__ void with_rank_count(int n, F &&f) {
     if constexpr (EXACT) f(FixedRanks<NR>{});
     else f(RankCount{n});
-}
-
-// Calls f(std::true_type{}) when every block scale of the unit takes the fast
-// quotient, else f(std::false_type{}).
-template <typename F>
-__device__ __forceinline__ void with_fast(bool fast, F &&f) {
-    if (fast) f(std::true_type{});
-    else f(std::false_type{});
 }
 
 // Elements of a 128-block that belong to this lane: 0..4.

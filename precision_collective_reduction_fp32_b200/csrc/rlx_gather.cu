@@ -12,9 +12,10 @@
 // conversion), so results are bit copies; a warp moves kUnroll x 512
 // contiguous bytes per step (lane l takes vectors l, l+32, ...), so each of
 // its stores to a destination row continues the previous one.  On the FP8
-// wire a warp handles kJ consecutive 128-element blocks at once (4 elements
-// per lane per block): it reads them, applies dequantise(quantise(.)) in
-// registers and writes every destination.
+// wire a warp handles J consecutive 128-element blocks at once (4 elements
+// per lane per block; J = 4 for fp32, 8 for the bf16 alltoall, see kJa2a):
+// it reads them, applies dequantise(quantise(.)) in registers and writes
+// every destination.
 // Units of work are numbered in memory order (segment-major) and handed out
 // in CTA-sized runs by for_each_unit, so the CTAs in flight stream one
 // compact stretch of the data.
@@ -88,7 +89,7 @@ ag_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t 
     });
 }
 
-// AllGather, FP8: unit = (source rank s, kJ blocks of its row); blocks
+// AllGather, FP8: unit = (source rank s, J blocks of its row); blocks
 // anchored at the row start.
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
@@ -96,23 +97,24 @@ ag_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, 
               FastDiv per_row) {
     const uint32_t units = per_row.d * static_cast<uint32_t>(n);
     const int e0 = lane_id() * 4;
+    constexpr int J = kJag<T>;
     for_each_unit<kPg>(units, [&](uint32_t g) {
         const uint32_t s = fast_div(g, per_row);
-        const size_t b0 = static_cast<size_t>(g - s * per_row.d) * kJ;
-        with_full((b0 + kJ) * kBlock <= m, [&](auto full) {
+        const size_t b0 = static_cast<size_t>(g - s * per_row.d) * J;
+        with_full((b0 + J) * kBlock <= m, [&](auto full) {
             const T *src = send + s * sstride + b0 * kBlock + e0;
-            float v[kJ][4];
-            int valid[kJ];
+            float v[J][4];
+            int valid[J];
 #pragma unroll
-            for (int j = 0; j < kJ; ++j) {
+            for (int j = 0; j < J; ++j) {
                 valid[j] = decltype(full)::value ? 4 : lane_valid((b0 + j) * kBlock, m);
                 load4<T, VEC>(src + j * kBlock, valid[j], v[j]);
             }
-            wire_fp8_blocks<kJ>(v);
+            wire_fp8_blocks<J>(v);
             for (int r = 0; r < n; ++r) {
                 T *dst = recv + r * rstride + s * m + b0 * kBlock + e0;
 #pragma unroll
-                for (int j = 0; j < kJ; ++j) store4<T, VEC>(dst + j * kBlock, valid[j], v[j]);
+                for (int j = 0; j < J; ++j) store4<T, VEC>(dst + j * kBlock, valid[j], v[j]);
             }
         });
     });
@@ -141,32 +143,33 @@ a2a_native_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t
     });
 }
 
-// AlltoAll, FP8: unit = (pair, kJ blocks); blocks anchored at the chunk start.
+// AlltoAll, FP8: unit = (pair, J blocks); blocks anchored at the chunk start.
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(kThreads)
 a2a_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, int n,
                FastDiv per_chunk, FastDiv ranks) {
     const uint32_t units = per_chunk.d * static_cast<uint32_t>(n) * static_cast<uint32_t>(n);
     const int e0 = lane_id() * 4;
+    constexpr int J = kJa2a<T>;
     for_each_unit<kPg>(units, [&](uint32_t g) {
         const uint32_t pair = fast_div(g, per_chunk);
         const uint32_t s = fast_div(pair, ranks), r = pair - s * ranks.d;
-        const size_t b0 = static_cast<size_t>(g - pair * per_chunk.d) * kJ;
-        with_full((b0 + kJ) * kBlock <= m, [&](auto full) {
+        const size_t b0 = static_cast<size_t>(g - pair * per_chunk.d) * J;
+        with_full((b0 + J) * kBlock <= m, [&](auto full) {
             const T *src = send + static_cast<size_t>(s) * sstride + static_cast<size_t>(r) * m +
                            b0 * kBlock + e0;
             T *dst = recv + static_cast<size_t>(r) * rstride + static_cast<size_t>(s) * m +
                      b0 * kBlock + e0;
-            float v[kJ][4];
-            int valid[kJ];
+            float v[J][4];
+            int valid[J];
 #pragma unroll
-            for (int j = 0; j < kJ; ++j) {
+            for (int j = 0; j < J; ++j) {
                 valid[j] = decltype(full)::value ? 4 : lane_valid((b0 + j) * kBlock, m);
                 load4<T, VEC>(src + j * kBlock, valid[j], v[j]);
             }
-            wire_fp8_blocks<kJ>(v);
+            wire_fp8_blocks<J>(v);
 #pragma unroll
-            for (int j = 0; j < kJ; ++j) store4<T, VEC>(dst + j * kBlock, valid[j], v[j]);
+            for (int j = 0; j < J; ++j) store4<T, VEC>(dst + j * kBlock, valid[j], v[j]);
         });
     });
 }
@@ -232,7 +235,7 @@ cudaError_t launch_all_gather(const void *send, size_t send_stride, void *recv,
         const T *s = static_cast<const T *>(send);
         T *r = static_cast<T *>(recv);
         const size_t nn = static_cast<size_t>(nranks);
-        const size_t per = wire == RLX_WIRE_NATIVE ? copy_units<T>(m) : block_units(m, kJ);
+        const size_t per = wire == RLX_WIRE_NATIVE ? copy_units<T>(m) : block_units(m, kJag<T>);
         if (!fits32(per)) return cudaErrorInvalidValue;
         const FastDiv fd = make_fastdiv(static_cast<uint32_t>(per));
         if (wire == RLX_WIRE_NATIVE)
@@ -250,7 +253,7 @@ cudaError_t launch_alltoall(const void *send, size_t send_stride, void *recv,
         const T *s = static_cast<const T *>(send);
         T *r = static_cast<T *>(recv);
         const size_t pairs = static_cast<size_t>(nranks) * static_cast<size_t>(nranks);
-        const size_t per = wire == RLX_WIRE_NATIVE ? copy_units<T>(m) : block_units(m, kJ);
+        const size_t per = wire == RLX_WIRE_NATIVE ? copy_units<T>(m) : block_units(m, kJa2a<T>);
         if (!fits32(per)) return cudaErrorInvalidValue;
         const FastDiv fd = make_fastdiv(static_cast<uint32_t>(per));
         const FastDiv fn = make_fastdiv(static_cast<uint32_t>(nranks));

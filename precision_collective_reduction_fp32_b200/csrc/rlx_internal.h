@@ -64,6 +64,14 @@ cudaError_t launch_tree_gather(void *recv, size_t count, size_t stride, int nran
                                const uint8_t *ws_codes, const float *ws_scales, bool vec,
                                cudaStream_t stream);
 
+// DDA-tree in one launch with chunk-ready counts (rlx_tree_fused.cu).
+// workspace: RLX_TREE_SYNC_BYTES of sync words (zero on entry), then on the
+// FP8 wire the payload.  status may be null.
+cudaError_t launch_tree_fused(const void *send, void *recv, size_t count, size_t stride,
+                              int nranks, size_t chunk, rlx_dtype dtype, rlx_wire wire,
+                              void *workspace, int *status, uint64_t limit_ns, bool vec,
+                              cudaStream_t stream);
+
 cudaError_t launch_reduce_scatter(const void *send, size_t send_stride, void *recv,
                                   size_t recv_stride, size_t m, int nranks, rlx_dtype dtype,
                                   rlx_wire wire, bool vec, cudaStream_t stream);

@@ -22,12 +22,8 @@ __device__ __forceinline__ void storev(T *p, int valid, const float (&v)[VecN<T>
             q.x = __float_as_uint(v[0]); q.y = __float_as_uint(v[1]);
             q.z = __float_as_uint(v[2]); q.w = __float_as_uint(v[3]);
         } else {
-            uint32_t w[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                w[k] = static_cast<uint32_t>(f32_to_bf16_bits(v[2 * k])) |
-                       (static_cast<uint32_t>(f32_to_bf16_bits(v[2 * k + 1])) << 16);
-            q = make_uint4(w[0], w[1], w[2], w[3]);
+            q = make_uint4(bf16x2_bits(v[0], v[1]), bf16x2_bits(v[2], v[3]),
+                           bf16x2_bits(v[4], v[5]), bf16x2_bits(v[6], v[7]));
         }
         st_stream(reinterpret_cast<uint4 *>(p), q);
     } else {
@@ -125,10 +121,12 @@ template <typename T> constexpr int kBpu = sizeof(T) == 2 ? RLX_BPU_BF16 : 1;
 
 // acc[j] = SUM_s wire(x_s) over the BPU adjacent 128-blocks at src + 128 j in
 // each of n rows, 4 elements per lane (valid[j] of them real; the rest +0).
-// Every (rank, block) pair is one FP8 block: its amax is one warp
-// reduction, and lane l computes the scale of pair l % (NR*BPU), which is
-// broadcast just before that pair is quantised.  The loads stay raw until
-// then, so a bf16 pair costs 2 registers.
+// Every (rank, block) pair is one FP8 block: its amax is one warp max
+// reduction of the lanes' amax keys, and lane l computes the scale of pair
+// l % (NR*BPU); the keys and the scales pass through the warp's
+// shared-memory slot (publish_scales), and each pair's scale is read from
+// there just before the pair is quantised.  The loads stay raw until then,
+// so a bf16 pair costs 2 registers.
 template <typename T, int NR, bool VEC, int BPU, typename N>
 __device__ __forceinline__ void reduce_blocks_fp8(const T *src, size_t pitch, N n,
                                                   const int (&valid)[BPU],
@@ -143,31 +141,35 @@ __device__ __forceinline__ void reduce_blocks_fp8(const T *src, size_t pitch, N 
         for (int j = 0; j < BPU; ++j)
             x[s][j] = s < n ? load_raw4<T, VEC>(src + s * pitch + j * kBlock + e0, valid[j])
                             : raw4_zero<T>();
-    const int mine = threadIdx.x & (K - 1);
-    uint32_t a = 0u;
+    // block (s, j) is pair s*BPU + j; its key goes to the slot as soon as the
+    // reduction gives it (four at a time)
+    begin_keys();
+    if constexpr (K % 4 == 0) {
 #pragma unroll
-    for (int s = 0; s < NR; ++s)
+        for (int k = 0; k < K; k += 4) {
+            uint32_t q[4];
 #pragma unroll
-        for (int j = 0; j < BPU; ++j) {
-            const uint32_t m = __reduce_max_sync(kFull, absmax4_bits(x[s][j]));
-            if (mine == s * BPU + j) a = m;
+            for (int i = 0; i < 4; ++i)
+                q[i] = __reduce_max_sync(kFull, amax_key(x[(k + i) / BPU][(k + i) % BPU]));
+            put_keys(k, q[0], q[1], q[2], q[3]);
         }
-    const Scale own = make_scale(__uint_as_float(a));
-    // one vote: when every scale of the unit takes the fast quotient (the
-    // usual case) the quantisation below is straight-line code the compiler
-    // can interleave across blocks
-    with_fast(RLX_FAST_VOTE && __all_sync(kFull, own.y != 0.0f), [&](auto fast) {
+    } else {
+#pragma unroll
+        for (int k = 0; k < K; ++k) put_key(k, __reduce_max_sync(kFull, amax_key(x[k / BPU][k % BPU])));
+    }
+    // when every scale of the unit takes the fast quotient (the usual case)
+    // the quantisation below is straight-line code the compiler can
+    // interleave across blocks
+    const bool fast = publish_scales<T, K>();
+    with_fast(RLX_FAST_VOTE && fast, [&](auto f) {
 #pragma unroll
         for (int s = 0; s < NR; ++s) {
             if (s < n) {
 #pragma unroll
                 for (int j = 0; j < BPU; ++j) {
-                    Scale sc;
-                    sc.s = __shfl_sync(kFull, own.s, s * BPU + j);
-                    sc.y = __shfl_sync(kFull, own.y, s * BPU + j);
                     float v[4];
                     widen4(x[s][j], v);
-                    wire4<decltype(fast)::value>(v, sc);
+                    wire4<decltype(f)::value>(v, scale_of(s * BPU + j));
                     if (s == 0) {
 #pragma unroll
                         for (int k = 0; k < 4; ++k) acc[j][k] = v[k];
@@ -183,13 +185,6 @@ __device__ __forceinline__ void reduce_blocks_fp8(const T *src, size_t pitch, N 
 }
 
 // ------------------------------------------------------ 16-byte bf16 stores
-
-// Two fp32 values -> two bf16 (round to nearest even) in one word, `lo` in the
-// low half.
-__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
-    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t *>(&h);
-}
 
 // Row pieces of 16 bytes for a bf16 block pair held as 4 values per lane per
 // block: lane 2i gets elements [8i, 8i+8) of block 0 and lane 2i+1 the same
@@ -256,8 +251,20 @@ __device__ __forceinline__ int vec_valid_in(size_t i0, size_t hi, Full) {
 #ifndef RLX_JD
 #define RLX_JD 8
 #endif
+// 128-blocks per warp unit of the single-source FP8 kernels with bf16 data
+// (alltoall, all-gather): more blocks than for fp32, since a bf16 block is
+// half the bytes and the per-unit work (indices, the scales' division) is
+// paid per unit
+#ifndef RLX_J_A2A_BF16
+#define RLX_J_A2A_BF16 8
+#endif
+#ifndef RLX_J_AG_BF16
+#define RLX_J_AG_BF16 4
+#endif
 constexpr int kUnroll = RLX_UNROLL;  // 16-byte vectors per lane in flight (native copies)
-constexpr int kJ = RLX_J;            // 128-blocks in flight per warp (FP8 single-source)
+constexpr int kJ = RLX_J;            // 128-blocks in flight per warp (FP8 single-source, fp32)
+template <typename T> constexpr int kJa2a = sizeof(T) == 2 ? RLX_J_A2A_BF16 : RLX_J;
+template <typename T> constexpr int kJag = sizeof(T) == 2 ? RLX_J_AG_BF16 : RLX_J;
 constexpr int kJd = RLX_JD;          // 128-blocks per warp when reading FP8 payloads
 
 template <typename T> constexpr int kV = 16 / sizeof(T);
@@ -394,12 +401,17 @@ __device__ __forceinline__ void tree_reduce_fp8_unit(uint32_t u, const T *send, 
             valid[j] = decltype(full)::value ? 4 : lane_valid(base + j * kBlock, count);
         float acc[BPU][4];
         reduce_blocks_fp8<T, NR, VEC, BPU>(send + base, stride, n, valid, acc);
-        float amax[BPU];
+        Scale2 sc[BPU];
+        if constexpr (BPU == 1) {
+            sc[0] = pack(make_scale(warp_amax4(acc[0])));
+        } else {
+            uint32_t key[BPU];
 #pragma unroll
-        for (int j = 0; j < BPU; ++j) amax[j] = warp_amax4(acc[j]);
-        Scale sc[BPU];
-        if constexpr (BPU == 1) sc[0] = make_scale(amax[0]);
-        else make_scales<BPU>(amax, sc);
+            for (int j = 0; j < BPU; ++j) key[j] = __float_as_uint(warp_amax4(acc[j]));
+            publish_scales<float, BPU>(key);
+#pragma unroll
+            for (int j = 0; j < BPU; ++j) sc[j] = scale_of(j);
+        }
 #pragma unroll
         for (int j = 0; j < BPU; ++j) {
             const size_t bj = base + j * kBlock;
@@ -407,7 +419,7 @@ __device__ __forceinline__ void tree_reduce_fp8_unit(uint32_t u, const T *send, 
                 const uint32_t codes = quant4(acc[j], sc[j]);
                 // default caching: pass 2 reads the payload back right away
                 *reinterpret_cast<uint32_t *>(ws_codes + bj + e0) = codes;
-                if (lane_id() == 0) ws_scales[bj / kBlock] = sc[j].s;
+                if (lane_id() == 0) ws_scales[bj / kBlock] = sc[j].s.x;
             }
         }
     });

@@ -52,37 +52,32 @@ quantize_kernel(const T *x, size_t rows, size_t n, size_t stride, uint8_t *codes
             uint8_t *cr = codes + row * stride + b0 * kBlock + e0;
             float v[kJq][4];
             int valid[kJq];
-            float amax[kJq];
+            uint32_t key[kJq];
 #pragma unroll
             for (int j = 0; j < kJq; ++j) {
                 valid[j] = F ? 4 : lane_valid((b0 + j) * kBlock, n);
                 load4<T, VEC>(xr + j * kBlock, valid[j], v[j]);
             }
 #pragma unroll
-            for (int j = 0; j < kJq; ++j) amax[j] = warp_amax4(v[j]);
-            Scale sc[kJq];
-            make_scales<kJq>(amax, sc);
+            for (int j = 0; j < kJq; ++j) key[j] = __float_as_uint(warp_amax4(v[j]));
+            with_fast(publish_scales<float, kJq>(key), [&](auto fast) {
 #pragma unroll
-            for (int j = 0; j < kJq; ++j) {
-                const uint32_t q = quant4(v[j], sc[j]);
-                uint8_t *dst = cr + j * kBlock;
-                if (VEC && valid[j] == 4) {
-                    st_stream(reinterpret_cast<unsigned int *>(dst), q);
-                } else {
+                for (int j = 0; j < kJq; ++j) {
+                    const uint32_t q = quant4<decltype(fast)::value>(v[j], scale_of(j));
+                    uint8_t *dst = cr + j * kBlock;
+                    if (VEC && valid[j] == 4) {
+                        st_stream(reinterpret_cast<unsigned int *>(dst), q);
+                    } else {
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        if (k < valid[j]) dst[k] = static_cast<uint8_t>(q >> (8 * k));
+                        for (int k = 0; k < 4; ++k)
+                            if (k < valid[j]) dst[k] = static_cast<uint8_t>(q >> (8 * k));
+                    }
                 }
-            }
+            });
             // lane j < kJq stores the scale of block b0 + j
             const int l = lane_id();
-            if (l < kJq && (F || b0 + l < nbr)) {
-                float s = sc[0].s;
-#pragma unroll
-                for (int j = 1; j < kJq; ++j)
-                    if (l == j) s = sc[j].s;
-                st_stream(scales + row * nbr + b0 + l, s);
-            }
+            if (l < kJq && (F || b0 + l < nbr))
+                st_stream(scales + row * nbr + b0 + l, scale_of(l).s.x);
         });
     });
 }

@@ -2,7 +2,10 @@
 // two Markstein corrections) with CUDA's IEEE division over every fp32 bit
 // pattern in [x_first, x_first + nx) and every scale given: the E4M3 codes of
 // the two quotients must always agree, and the quotients themselves bit for
-// bit wherever |x/s| >= 2^-12 (below that every code is +-0).
+// bit wherever |x/s| >= 2^-12 (below that every code is +-0).  Both forms are
+// checked: the scalar quotient_rn, and the packed negated quotient the
+// kernels use (neg_quotient2, whose result must be exactly -quotient_rn's,
+// and whose sign-flipped codes must be the IEEE quotient's codes).
 // Built and loaded by tests/test_gpu_quotient.py; not part of the library.
 #include <cstdint>
 #include <cstdio>
@@ -17,11 +20,18 @@ __global__ void quotient_check_kernel(const float *scales, int ns, uint32_t x_fi
         const float x = __uint_as_float(x_first + static_cast<uint32_t>(i));
         for (int k = 0; k < ns; ++k) {
             const float s = scales[k];
-            const float q = rlx::quotient_rn(x, s, __frcp_rn(s));
+            const float y = __frcp_rn(s);
+            const float q = rlx::quotient_rn(x, s, y);
+            const rlx::Scale2 sc = rlx::pack(rlx::Scale{s, -y});
+            const float2 p = rlx::neg_quotient2(make_float2(x, -x), sc);   // -q(x), -q(-x)
             const float ref = __fdiv_rn(x, s);
             const bool bits_matter = fabsf(ref) >= 0x1p-12f;
+            const uint32_t ref_code = rlx::e4m3x2_from_f32(ref, -ref);
             const bool differ = (bits_matter && __float_as_uint(q) != __float_as_uint(ref)) ||
-                                rlx::e4m3x2_from_f32(q, 0.0f) != rlx::e4m3x2_from_f32(ref, 0.0f);
+                                (bits_matter && __float_as_uint(p.x) != (__float_as_uint(ref) ^ 0x80000000u)) ||
+                                (bits_matter && __float_as_uint(p.y) != __float_as_uint(ref)) ||
+                                rlx::e4m3x2_from_f32(q, -q) != ref_code ||
+                                (rlx::e4m3x2_from_f32(p.x, p.y) ^ 0x8080u) != ref_code;
             if (differ) {
                 if (atomicAdd(mismatches, 1ull) == 0ull) {
                     witness[0] = __float_as_uint(x);

@@ -53,6 +53,10 @@ def test_workspace_bytes(L):
     assert f(B.RLX_COLL_ALLREDUCE_TREE, 1000, 8, B.RLX_F32, B.RLX_WIRE_NATIVE) == 0
     assert f(B.RLX_COLL_ALLREDUCE_TREE, 1000, 1, B.RLX_F32, B.RLX_WIRE_FP8_E4M3) == 0
     assert f(B.RLX_COLL_ALLREDUCE_FLAT, 1000, 8, B.RLX_F32, B.RLX_WIRE_FP8_E4M3) == 0
+    # the one-launch tree: sync words, then the FP8 payload
+    assert f(B.RLX_COLL_ALLREDUCE_TREE_FUSED, 1000, 8, B.RLX_F32, B.RLX_WIRE_NATIVE) == 256
+    assert f(B.RLX_COLL_ALLREDUCE_TREE_FUSED, 1000, 8, B.RLX_F32, B.RLX_WIRE_FP8_E4M3) == 256 + 1280
+    assert f(B.RLX_COLL_ALLREDUCE_TREE_FUSED, 1000, 1, B.RLX_F32, B.RLX_WIRE_FP8_E4M3) == 0
 
 
 def _st(name, *args):
@@ -162,3 +166,22 @@ def test_build_flags_keep_ieee_rounding():
         assert flag in f
     assert "arch=compute_100a,code=sm_100a" in f
     assert not any(x.startswith("--use_fast_math") or x == "-use_fast_math" for x in f)
+
+
+def test_fused_tree_rejects_before_launch(L):
+    """Bad arguments and bad workspaces of rlx_allreduce_tree_fused come back
+    as status codes before anything is launched."""
+    F, FP8, NAT = B.RLX_F32, B.RLX_WIRE_FP8_E4M3, B.RLX_WIRE_NATIVE
+    need = B.rlx_workspace_bytes(B.RLX_COLL_ALLREDUCE_TREE_FUSED, 1000, 8, F, FP8)
+    ws, st = A + 4 * Z, A + 5 * Z
+    call = lambda *a: _st("rlx_allreduce_tree_fused", *a)
+    assert call(A, A + Z, 1000, 1000, 8, F, FP8, B.RLX_SUM, None, 0, st, 0, None) == B.RLX_ERR_WORKSPACE
+    assert call(A, A + Z, 1000, 1000, 8, F, FP8, B.RLX_SUM, ws, need - 1, st, 0, None) == B.RLX_ERR_WORKSPACE
+    assert call(A, A + Z, 1000, 1000, 8, F, NAT, B.RLX_SUM, ws + 8, 256, st, 0, None) == B.RLX_ERR_WORKSPACE
+    assert call(A, A + Z, 1000, 1000, 8, F, FP8, B.RLX_SUM, A + 16, need, st, 0, None) == B.RLX_ERR_WORKSPACE
+    assert call(A, A + Z, 1000, 1000, 8, F, FP8, B.RLX_SUM, ws, need, st + 2, 0, None) == B.RLX_ERR_ALIGNMENT
+    assert call(A, A + Z, 1000, 1000, 8, F, FP8, B.RLX_SUM, ws, need, A + 64, 0, None) == B.RLX_ERR_INVALID_ARG
+    assert call(A, A + Z, 1000, 1000, 8, F, FP8, 1, ws, need, st, 0, None) == B.RLX_ERR_UNSUPPORTED
+    assert call(A, A + Z, 1000, 999, 8, F, FP8, B.RLX_SUM, ws, need, st, 0, None) == B.RLX_ERR_INVALID_ARG
+    assert call(A, A + Z, 1000, 1000, 17, F, FP8, B.RLX_SUM, ws, need, st, 0, None) == B.RLX_ERR_INVALID_ARG
+    assert call(None, A + Z, 1000, 1000, 8, F, FP8, B.RLX_SUM, ws, need, st, 0, None) == B.RLX_ERR_INVALID_ARG
