@@ -261,31 +261,67 @@ static_assert(kQuotient >= 0 && kQuotient <= 2, "RLX_QUOTIENT must be 0, 1 or 2"
 // -fl32(448 / amax); RLX_QUOTIENT=2: ny = 0, every element takes the IEEE
 // division.)  The reciprocal is kept negated because the quantiser works on
 // the negated quotient (see neg_quotient2).
+// 1: the quotient starts from a two-term reciprocal (see neg_quotient2),
+// which saves one of its five packed steps; 0: the plain reciprocal and two
+// corrections.
+#ifndef RLX_QUOTIENT_2TERM
+#define RLX_QUOTIENT_2TERM 0
+#endif
+constexpr bool k2Term = RLX_QUOTIENT_2TERM && kQuotient == 0;
+
+// With the two-term reciprocal the scale also carries nlo = -y_lo, where
+// y_hi = RD(1/s) and y_lo = RN((1 - s*y_hi) * y) >= +0 (so nlo <= -0).
 struct Scale {
-    float s, ny;
+    float s, ny, nhi, nlo;
 };
-__device__ __forceinline__ Scale make_scale(float amax) {
+// The reciprocal terms of a scale s for the correctly rounded quotient.
+__device__ __forceinline__ Scale reciprocal_terms(float s) {
     Scale r;
-    r.s = __fdiv_rn(amax, kE4m3Max);
-    if constexpr (kQuotient == 0) r.ny = r.s >= kMinFastScale ? -__frcp_rn(r.s) : 0.0f;
-    else if constexpr (kQuotient == 1) r.ny = r.s >= kMinFastScale ? -__fdiv_rn(kE4m3Max, amax) : 0.0f;
-    else r.ny = 0.0f;
+    r.s = s;
+    r.nhi = r.nlo = 0.0f;
+    r.ny = s >= kMinFastScale ? -__frcp_rn(s) : 0.0f;
+    if constexpr (k2Term) {
+        if (r.ny != 0.0f) {
+            const float hi = __frcp_rd(s);
+            // 1 - s*hi is exact (hi is a faithful reciprocal) and >= 0
+            const float e = __fmaf_rn(-s, hi, 1.0f);
+            r.nhi = -hi;
+            r.nlo = -__fmul_rn(e, -r.ny);
+        }
+    }
     return r;
 }
 
-// A block scale as the packed two-lane instructions take it: (s, s) and
-// (ny, ny) in adjacent registers.
+__device__ __forceinline__ Scale make_scale(float amax) {
+    Scale r;
+    r.s = __fdiv_rn(amax, kE4m3Max);
+    r.nhi = r.nlo = 0.0f;
+    if constexpr (kQuotient == 0) {
+        r = reciprocal_terms(r.s);
+    } else if constexpr (kQuotient == 1) {
+        r.ny = r.s >= kMinFastScale ? -__fdiv_rn(kE4m3Max, amax) : 0.0f;
+    } else {
+        r.ny = 0.0f;
+    }
+    return r;
+}
+
+// A block scale as the packed two-lane instructions take it: (s, s),
+// (ny, ny) (and (nhi, nhi), (nlo, nlo)) in adjacent registers.
 struct Scale2 {
-    float2 s, ny;
+    float2 s, ny, nhi, nlo;
 };
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
-__device__ __forceinline__ Scale2 pack(Scale sc) { return {f2(sc.s, sc.s), f2(sc.ny, sc.ny)}; }
+__device__ __forceinline__ Scale2 pack(Scale sc) {
+    return {f2(sc.s, sc.s), f2(sc.ny, sc.ny), f2(sc.nhi, sc.nhi), f2(sc.nlo, sc.nlo)};
+}
 
 // Per-warp shared memory through which the lanes of a warp exchange block
 // amaxes and scales (a slot per warp of the 256-thread CTA).
 constexpr int kWarpsPerCta = 8;
 struct alignas(16) WarpScratch {
     float4 scale[32];   // block k: (s, s, ny, ny)
+    float4 split[k2Term ? 32 : 1];   // block k: (nhi, nhi, nlo, nlo) (two-term reciprocal)
     uint32_t key[32];   // block k: its amax key
 };
 __device__ __forceinline__ WarpScratch &warp_scratch() {
@@ -321,7 +357,10 @@ __device__ __forceinline__ bool publish_scales() {
     const int lane = threadIdx.x & 31;
     __syncwarp();
     const Scale own = make_scale(amax_of<T>(w.key[lane & (K - 1)]));
-    if (lane < K) w.scale[lane] = make_float4(own.s, own.s, own.ny, own.ny);
+    if (lane < K) {
+        w.scale[lane] = make_float4(own.s, own.s, own.ny, own.ny);
+        if constexpr (k2Term) w.split[lane] = make_float4(own.nhi, own.nhi, own.nlo, own.nlo);
+    }
     const bool fast = __all_sync(kFull, own.ny != 0.0f);
     __syncwarp();
     return fast;
@@ -341,7 +380,11 @@ __device__ __forceinline__ bool publish_scales(const uint32_t (&key)[K]) {
 }
 __device__ __forceinline__ Scale2 scale_of(int k) {
     const float4 v = warp_scratch().scale[k];
-    return {f2(v.x, v.y), f2(v.z, v.w)};
+    if constexpr (k2Term) {
+        const float4 u = warp_scratch().split[k];
+        return {f2(v.x, v.y), f2(v.z, v.w), f2(u.x, u.y), f2(u.z, u.w)};
+    }
+    return {f2(v.x, v.y), f2(v.z, v.w), f2(0.0f, 0.0f), f2(0.0f, 0.0f)};
 }
 
 // fl32(x / s), correctly rounded, from y = fl32(1/s) (s >= 2^-90).
@@ -381,8 +424,20 @@ __device__ __forceinline__ float quotient_rn(float x, float s, float y) {
 // to +0 this one does too, which leaves p = -q intact since q != 0 there;
 // x = +-0 gives p = -+0.  No operand needs a per-element negation.
 // (RLX_QUOTIENT=1: p = x * ny.)
+// Two-term form (RLX_QUOTIENT_2TERM): y_hi = RD(1/s) and y_lo =
+// RN((1 - s*y_hi) * y) approximate 1/s to about 2^-47, so
+// q0 = RN(x*y_hi + RN(x*y_lo)) is already faithful and one Markstein step
+// rounds it correctly: four packed steps instead of five.  Negated as
+// above; since -y_lo is never +0, x*(-y_lo) has the sign of -x when x is a
+// zero, and p0 = -+0 for x = +-0 as required.
 __device__ __forceinline__ float2 neg_quotient2(float2 x, const Scale2 &sc) {
 #if RLX_PACKED_F32X2
+    if constexpr (k2Term) {
+        const float2 t = __fmul2_rn(x, sc.nlo);
+        float2 p = __ffma2_rn(x, sc.nhi, t);    // -RN(x*y_hi + x*y_lo), faithful
+        const float2 r = __ffma2_rn(sc.s, p, x);
+        return __ffma2_rn(r, sc.ny, p);
+    }
     float2 p = __fmul2_rn(x, sc.ny);
     if constexpr (kQuotient == 1) return p;
     float2 r = __ffma2_rn(sc.s, p, x);   // s*p + x = -(s*q - x)

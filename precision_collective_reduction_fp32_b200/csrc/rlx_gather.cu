@@ -13,7 +13,7 @@
 // contiguous bytes per step (lane l takes vectors l, l+32, ...), so each of
 // its stores to a destination row continues the previous one.  On the FP8
 // wire a warp handles J consecutive 128-element blocks at once (4 elements
-// per lane per block; J = 4 for fp32, 8 for the bf16 alltoall, see kJa2a):
+// per lane per block; J per element type, see kJa2a and kJag):
 // it reads them, applies dequantise(quantise(.)) in registers and writes
 // every destination.
 // Units of work are numbered in memory order (segment-major) and handed out

@@ -252,11 +252,11 @@ __device__ __forceinline__ int vec_valid_in(size_t i0, size_t hi, Full) {
 #define RLX_JD 8
 #endif
 // 128-blocks per warp unit of the single-source FP8 kernels with bf16 data
-// (alltoall, all-gather): more blocks than for fp32, since a bf16 block is
-// half the bytes and the per-unit work (indices, the scales' division) is
-// paid per unit
+// (alltoall, all-gather).  8 blocks per alltoall unit halve the per-unit work
+// (indices, the scales' division) but measured slower in the library at the
+// prefill size (231 against 223 us), so both stay at 4.
 #ifndef RLX_J_A2A_BF16
-#define RLX_J_A2A_BF16 8
+#define RLX_J_A2A_BF16 4
 #endif
 #ifndef RLX_J_AG_BF16
 #define RLX_J_AG_BF16 4

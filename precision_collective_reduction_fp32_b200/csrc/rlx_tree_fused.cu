@@ -11,9 +11,10 @@
 // fetches a peer's chunk once the peer's ready flag is up:
 //
 //   * work queue: the kernel's work is cut into CTA-sized runs of units (the
-//     unit bodies of the two-pass kernels, rlx_passes.cuh); tickets
-//     0 .. R1-1 are reduce-scatter (pass 1) runs, R1 .. R1+R2-1 all-gather
-//     (pass 2) runs, and a CTA takes its next ticket from one atomic counter;
+//     unit bodies of the two-pass kernels, rlx_passes.cuh): tickets 0 .. R1-1
+//     are reduce-scatter (pass 1) runs, R1 .. R1+R2-1 all-gather (pass 2)
+//     runs, each in memory order (rlx_tree_plan.cuh), and a CTA takes its
+//     next ticket from one atomic counter while its current run executes;
 //   * chunk-ready counts: after a pass-1 run the CTA adds, with release
 //     semantics, how many pass-1 units (native) or 128-blocks (FP8) of each
 //     chunk it finished to that chunk's count;
@@ -24,9 +25,10 @@
 //     the failure, skips the work that depended on the wait, and returns.
 //
 // Why no CTA can wait forever: tickets are handed out in order, and only to
-// CTAs that are running, so a CTA holds a pass-2 ticket only after every
-// pass-1 ticket went to a running CTA; pass-1 work never waits, so every
-// count a pass-2 warp waits for is eventually reached, however many CTAs are
+// CTAs that are running, and every pass-1 run has an earlier ticket than
+// every pass-2 run; so a CTA holds a pass-2 ticket only after all pass-1
+// work went to running CTAs.  Pass-1 work never waits, so every count a
+// pass-2 warp waits for is eventually reached, however many CTAs are
 // resident and in whatever order the hardware starts them.
 //
 // Exit: every CTA counts itself done; the last one clears the ticket, the
@@ -36,7 +38,7 @@
 #include <map>
 #include <mutex>
 
-#include "rlx_passes.cuh"
+#include "rlx_tree_plan.cuh"
 
 namespace rlx {
 namespace {
@@ -106,68 +108,49 @@ struct FusedArgs {
     const void *send;
     void *recv;
     size_t count, stride, chunk;
-    int n;
     uint8_t *ws_codes;
     float *ws_scales;
     TreeSync *sync;
     int *status;
     uint64_t limit_ns;
-    uint32_t runs1, runs2;        // pass-1 / pass-2 runs
-    uint32_t units1, units2;      // pass-1 / pass-2 units
-    FastDiv per1, per2;           // native: pass-1 / pass-2 units per chunk
-    uint32_t blocks_per_chunk;    // FP8: 128-blocks per chunk
-    uint32_t nblk;                // FP8: 128-blocks in count
+    TreePlan plan;
 };
 
-// Units per warp in one run.
-constexpr int kRunP = 1;
-constexpr uint32_t kRunUnits = kWarpsPerCta * kRunP;
-
-// Total pass-1 work of chunk c: native units, or 128-blocks on the FP8 wire.
-template <bool FP8>
-__device__ __forceinline__ uint32_t chunk_target(const FusedArgs &a, uint32_t c) {
-    if constexpr (!FP8) {
-        return a.per1.d;
-    } else {
-        const uint32_t lo = c * a.blocks_per_chunk;
-        if (lo >= a.nblk) return 0;
-        const uint32_t rem = a.nblk - lo;
-        return rem < a.blocks_per_chunk ? rem : a.blocks_per_chunk;
-    }
-}
-
-// The kernel holds both passes' unit bodies; two resident CTAs per SM (up to
-// 128 registers a thread) keep both free of spills, and one wave of them
-// covers the small messages this form is for.
 template <typename T, int NR, bool VEC, bool EXACT, bool FP8>
 __global__ void __launch_bounds__(kThreads, NR <= 8 ? 2 : 1)
 tree_fused_kernel(FusedArgs a) {
-    __shared__ uint32_t s_ticket;
+    __shared__ uint32_t s_ticket[2];
     __shared__ uint32_t s_done[RLX_MAX_RANKS];
     pdl_begin();
     const int lane = lane_id();
     const uint32_t warp = threadIdx.x >> 5;
-    const uint32_t total = a.runs1 + a.runs2;
+    const TreePlan &pl = a.plan;
+    const uint32_t total = pl.runs1 + pl.runs2;
     uint32_t ready_mask = 0;   // chunks this warp has seen complete
     bool failed = false;
-    with_rank_count<NR, EXACT>(a.n, [&](auto nn) {
-        for (;;) {
-            if (threadIdx.x == 0) s_ticket = atomicAdd(&a.sync->ticket, 1u);
+    if (threadIdx.x == 0) s_ticket[0] = atomicAdd(&a.sync->ticket, 1u);
+    with_rank_count<NR, EXACT>(static_cast<int>(pl.n), [&](auto nn) {
+        for (uint32_t round = 0;; ++round) {
             if (threadIdx.x < RLX_MAX_RANKS) s_done[threadIdx.x] = 0;
             __syncthreads();
-            const uint32_t t = s_ticket;
+            const uint32_t t = s_ticket[round & 1];
             if (t >= total) break;
-            if (t < a.runs1) {
-                // ---- pass 1: reduce-scatter units of run t
-#pragma unroll 1
-                for (int p = 0; p < kRunP; ++p) {
-                    const uint32_t g = t * kRunUnits + p * kWarpsPerCta + warp;
-                    if (g >= a.units1) continue;
+            // the next ticket is fetched while this run executes, so the round
+            // trip to the counter is off the critical path (a ticket is still
+            // only handed to a running CTA, which finishes its current run
+            // before it can wait on anything)
+            if (threadIdx.x == 0) s_ticket[(round + 1) & 1] = atomicAdd(&a.sync->ticket, 1u);
+            bool pass2;
+            const uint32_t run = plan_resolve(pl, t, &pass2);   // same in every thread
+            const uint32_t g = run * kRunUnits + warp;          // this warp's unit
+            if (!pass2) {
+                // ---- pass 1: reduce-scatter unit g
+                if (g < pl.units1) {
                     if constexpr (!FP8) {
                         tree_reduce_native_unit<T, NR, VEC>(g, static_cast<const T *>(a.send),
                                                             static_cast<T *>(a.recv), a.count,
-                                                            a.stride, nn, a.chunk, a.per1);
-                        if (lane == 0) atomicAdd(&s_done[fast_div(g, a.per1)], 1u);
+                                                            a.stride, nn, a.chunk, pl.per1);
+                        if (lane == 0) atomicAdd(&s_done[fast_div(g, pl.per1)], 1u);
                     } else {
                         tree_reduce_fp8_unit<T, NR, VEC>(g, static_cast<const T *>(a.send), a.count,
                                                          a.stride, nn, a.ws_codes, a.ws_scales);
@@ -176,7 +159,7 @@ tree_fused_kernel(FusedArgs a) {
 #pragma unroll
                             for (uint32_t j = 0; j < B; ++j) {
                                 const uint32_t b = g * B + j;
-                                if (b < a.nblk) atomicAdd(&s_done[b / a.blocks_per_chunk], 1u);
+                                if (b < pl.nblk) atomicAdd(&s_done[fast_div(b, pl.chunk_blocks)], 1u);
                             }
                         }
                     }
@@ -184,47 +167,34 @@ tree_fused_kernel(FusedArgs a) {
                 __syncthreads();
                 // publish: the CTA's writes (ordered before this thread by the
                 // barrier) become visible before the count does
-                if (threadIdx.x < static_cast<unsigned>(a.n) && s_done[threadIdx.x] != 0)
+                if (threadIdx.x < pl.n && s_done[threadIdx.x] != 0)
                     red_release_add(&a.sync->ready[threadIdx.x], s_done[threadIdx.x]);
-            } else {
-                // ---- pass 2: all-gather units of run t - runs1
-                const uint32_t t2 = t - a.runs1;
-#pragma unroll 1
-                for (int p = 0; p < kRunP; ++p) {
-                    const uint32_t g = t2 * kRunUnits + p * kWarpsPerCta + warp;
-                    if (g >= a.units2 || failed) continue;
-                    // the chunks this unit reads
-                    uint32_t c_lo, c_hi;
-                    if constexpr (!FP8) {
-                        c_lo = c_hi = fast_div(g, a.per2);
-                    } else {
-                        const uint32_t b0 = g * kJd;
-                        const uint32_t b1 = min(b0 + kJd, a.nblk) - 1;
-                        c_lo = b0 / a.blocks_per_chunk;
-                        c_hi = b1 / a.blocks_per_chunk;
-                    }
-                    // lane 0 waits (acquire); the warp barrier orders the
-                    // other lanes' reads of the chunk after it
-                    for (uint32_t c = c_lo; c <= c_hi && !failed; ++c) {
-                        if (ready_mask & (1u << c)) continue;
-                        int ok = 1;
-                        if (lane == 0) ok = wait_chunk(a.sync, c, chunk_target<FP8>(a, c), a.limit_ns);
-                        if (__shfl_sync(kFull, ok, 0))
-                            ready_mask |= 1u << c;
-                        else
-                            failed = true;
-                    }
-                    __syncwarp();
-                    if (failed) continue;
+            } else if (g < pl.units2 && !failed) {
+                // ---- pass 2: all-gather unit g, once the chunks it reads are ready
+                uint32_t c_lo, c_hi;
+                plan_pass2_chunks(pl, g, &c_lo, &c_hi);
+                // lane 0 waits (acquire); the warp barrier orders the other
+                // lanes' reads of the chunk after it
+                for (uint32_t c = c_lo; c <= c_hi && !failed; ++c) {
+                    if (ready_mask & (1u << c)) continue;
+                    int ok = 1;
+                    if (lane == 0) ok = wait_chunk(a.sync, c, plan_chunk_target(pl, c), a.limit_ns);
+                    if (__shfl_sync(kFull, ok, 0))
+                        ready_mask |= 1u << c;
+                    else
+                        failed = true;
+                }
+                __syncwarp();
+                if (!failed) {
                     if constexpr (!FP8)
                         tree_gather_native_unit<T, VEC>(g, static_cast<T *>(a.recv), a.count, a.stride,
-                                                        a.n, a.chunk, a.per2);
+                                                        static_cast<int>(pl.n), a.chunk, pl.per2);
                     else
                         tree_gather_fp8_unit<T, VEC>(g, static_cast<T *>(a.recv), a.count, a.stride,
-                                                     a.n, a.ws_codes, a.ws_scales);
+                                                     static_cast<int>(pl.n), a.ws_codes, a.ws_scales);
                 }
             }
-            __syncthreads();   // s_ticket and s_done are rewritten next round
+            __syncthreads();   // s_done is rewritten next round, s_ticket[round & 1] the one after
         }
     });
     // ---- exit: the last CTA out clears the sync words and reports
@@ -289,45 +259,24 @@ cudaError_t launch_tree_fused(const void *send, void *recv, size_t count, size_t
     a.count = count;
     a.stride = stride;
     a.chunk = chunk;
-    a.n = nranks;
     a.sync = static_cast<TreeSync *>(workspace);
     a.status = status;
     a.limit_ns = limit_ns;
-    const size_t nblk = (count + kBlock - 1) / kBlock;
-    if (wire == RLX_WIRE_FP8_E4M3) {
+    const bool fp8 = wire == RLX_WIRE_FP8_E4M3;
+    if (fp8) {
+        const size_t nblk = (count + kBlock - 1) / kBlock;
         a.ws_codes = static_cast<uint8_t *>(workspace) + RLX_TREE_SYNC_BYTES;
         a.ws_scales = reinterpret_cast<float *>(a.ws_codes + nblk * kBlock);
     }
     return dispatch_fused(dtype, nranks, vec, [&]<typename T, int NR, bool VEC, bool EX>() {
-        size_t units1, units2;
-        if (wire == RLX_WIRE_NATIVE) {
-            const size_t per1 = tree_reduce_native_per_chunk<T>(chunk);
-            const size_t per2 = tree_gather_native_per_chunk<T>(chunk);
-            units1 = per1 * static_cast<size_t>(nranks);
-            units2 = per2 * static_cast<size_t>(nranks);
-            if (units1 >= (size_t{1} << 31) || units2 >= (size_t{1} << 31)) return cudaErrorInvalidValue;
-            a.per1 = make_fastdiv(static_cast<uint32_t>(per1));
-            a.per2 = make_fastdiv(static_cast<uint32_t>(per2));
-        } else {
-            units1 = (nblk + kBpu<T> - 1) / kBpu<T>;
-            units2 = tree_gather_fp8_units(count);
-            if (nblk >= (size_t{1} << 31)) return cudaErrorInvalidValue;
-            a.blocks_per_chunk = static_cast<uint32_t>(chunk / kBlock);
-            a.nblk = static_cast<uint32_t>(nblk);
-        }
-        a.units1 = static_cast<uint32_t>(units1);
-        a.units2 = static_cast<uint32_t>(units2);
-        a.runs1 = static_cast<uint32_t>((units1 + kRunUnits - 1) / kRunUnits);
-        a.runs2 = static_cast<uint32_t>((units2 + kRunUnits - 1) / kRunUnits);
-        const void *k = wire == RLX_WIRE_NATIVE
-                            ? reinterpret_cast<const void *>(tree_fused_kernel<T, NR, VEC, EX, false>)
-                            : reinterpret_cast<const void *>(tree_fused_kernel<T, NR, VEC, EX, true>);
+        if (!make_tree_plan<T>(count, nranks, chunk, fp8, &a.plan)) return cudaErrorInvalidValue;
+        const void *k = !fp8 ? reinterpret_cast<const void *>(tree_fused_kernel<T, NR, VEC, EX, false>)
+                             : reinterpret_cast<const void *>(tree_fused_kernel<T, NR, VEC, EX, true>);
         const int resident = resident_ctas(k);
         if (resident <= 0) return cudaErrorInvalidValue;
-        const size_t runs = static_cast<size_t>(a.runs1) + a.runs2;
+        const size_t runs = static_cast<size_t>(a.plan.runs1) + a.plan.runs2;
         const dim3 grid(static_cast<unsigned>(runs < static_cast<size_t>(resident) ? runs : resident));
-        if (wire == RLX_WIRE_NATIVE)
-            return launch_kernel(tree_fused_kernel<T, NR, VEC, EX, false>, grid, stream, a);
+        if (!fp8) return launch_kernel(tree_fused_kernel<T, NR, VEC, EX, false>, grid, stream, a);
         return launch_kernel(tree_fused_kernel<T, NR, VEC, EX, true>, grid, stream, a);
     });
 }

@@ -5,7 +5,9 @@
 // bit wherever |x/s| >= 2^-12 (below that every code is +-0).  Both forms are
 // checked: the scalar quotient_rn, and the packed negated quotient the
 // kernels use (neg_quotient2, whose result must be exactly -quotient_rn's,
-// and whose sign-flipped codes must be the IEEE quotient's codes).
+// and whose sign-flipped codes must be the IEEE quotient's codes) -- in
+// whichever form the build selects (RLX_QUOTIENT_2TERM: the two-term
+// reciprocal and one correction, else two corrections).
 // Built and loaded by tests/test_gpu_quotient.py; not part of the library.
 #include <cstdint>
 #include <cstdio>
@@ -22,7 +24,7 @@ __global__ void quotient_check_kernel(const float *scales, int ns, uint32_t x_fi
             const float s = scales[k];
             const float y = __frcp_rn(s);
             const float q = rlx::quotient_rn(x, s, y);
-            const rlx::Scale2 sc = rlx::pack(rlx::Scale{s, -y});
+            const rlx::Scale2 sc = rlx::pack(rlx::reciprocal_terms(s));
             const float2 p = rlx::neg_quotient2(make_float2(x, -x), sc);   // -q(x), -q(-x)
             const float ref = __fdiv_rn(x, s);
             const bool bits_matter = fabsf(ref) >= 0x1p-12f;
