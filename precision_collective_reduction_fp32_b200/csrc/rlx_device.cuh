@@ -263,7 +263,10 @@ static_assert(kQuotient >= 0 && kQuotient <= 2, "RLX_QUOTIENT must be 0, 1 or 2"
 // the negated quotient (see neg_quotient2).
 // 1: the quotient starts from a two-term reciprocal (see neg_quotient2),
 // which saves one of its five packed steps; 0: the plain reciprocal and two
-// corrections.
+// corrections.  Both give the correctly rounded quotient (the quotient test
+// checks both); the two-term form measured slower (bf16 tree pass 1 at a
+// quarter of the prefill size: 43.3 against 39.8 us -- the second scale
+// load and the extra registers cost more than the step saves), so it is off.
 #ifndef RLX_QUOTIENT_2TERM
 #define RLX_QUOTIENT_2TERM 0
 #endif

@@ -20,14 +20,17 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "cuda", "quotient_check.cu")
 
 
-@pytest.fixture(scope="module")
-def qlib(tmp_path_factory):
+# both forms of the packed quotient: two Markstein corrections, and the
+# two-term reciprocal with one correction
+@pytest.fixture(scope="module", params=["two_corrections", "two_term_reciprocal"])
+def qlib(request, tmp_path_factory):
     import torch
     assert torch.cuda.is_available()
     so = str(tmp_path_factory.mktemp("qcheck") / "libqcheck.so")
+    form = ["-DRLX_QUOTIENT_2TERM=1"] if request.param == "two_term_reciprocal" else []
     subprocess.check_call(["/usr/local/cuda/bin/nvcc", "-gencode", "arch=compute_100a,code=sm_100a",
                            "-O3", "-std=c++20", "-fmad=false", "-Xcompiler", "-fPIC", "-shared",
-                           "-o", so, SRC])
+                           *form, "-o", so, SRC])
     L = ctypes.CDLL(so)
     L.quotient_check.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_uint32, ctypes.c_uint32,
                                  ctypes.c_void_p, ctypes.c_void_p]
