@@ -111,6 +111,8 @@ ag_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m, 
                 load4<T, VEC>(src + j * kBlock, valid[j], v[j]);
             }
             wire_fp8_blocks<J>(v);
+            // row by row: all J blocks of a row before the next row (storing
+            // each block to every row in turn measured 5 % slower)
             for (int r = 0; r < n; ++r) {
                 T *dst = recv + r * rstride + s * m + b0 * kBlock + e0;
 #pragma unroll
@@ -160,16 +162,13 @@ a2a_fp8_kernel(const T *send, size_t sstride, T *recv, size_t rstride, size_t m,
                            b0 * kBlock + e0;
             T *dst = recv + static_cast<size_t>(r) * rstride + static_cast<size_t>(s) * m +
                      b0 * kBlock + e0;
-            float v[J][4];
             int valid[J];
 #pragma unroll
-            for (int j = 0; j < J; ++j) {
+            for (int j = 0; j < J; ++j)
                 valid[j] = decltype(full)::value ? 4 : lane_valid((b0 + j) * kBlock, m);
-                load4<T, VEC>(src + j * kBlock, valid[j], v[j]);
-            }
-            wire_fp8_blocks<J>(v);
-#pragma unroll
-            for (int j = 0; j < J; ++j) store4<T, VEC>(dst + j * kBlock, valid[j], v[j]);
+            wire_blocks_raw<T, VEC, J>(src, valid, [&](int j, const float (&v)[4]) {
+                store4<T, VEC>(dst + j * kBlock, valid[j], v);
+            });
         });
     });
 }

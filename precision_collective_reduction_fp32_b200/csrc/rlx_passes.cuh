@@ -184,6 +184,72 @@ __device__ __forceinline__ void reduce_blocks_fp8(const T *src, size_t pitch, N 
     });
 }
 
+// ------------------------------------------------ FP8 wire, one sender's blocks
+
+// What the receiver of one sender holds after J consecutive 128-blocks of it
+// crossed the FP8 wire: the warp loads block j at src + 128 j (4 elements
+// per lane, valid[j] of them real; the rest +0), finds each block's amax by
+// one max reduction of the lanes' amax keys (passed to the warp's
+// shared-memory slot four at a time), and then widens, quantises and
+// dequantises one block at a time, handing it to emit(j, v) (which stores
+// it).  The loads stay raw until their block is converted, so a bf16 block
+// holds 2 registers until then instead of 4.
+// The scales of the J blocks held raw in x, made known to the warp
+// (publish_scales); true when every block takes the fast quotient.
+template <typename T, int J>
+__device__ __forceinline__ bool scales_of_raw_blocks(const Raw4<T> (&x)[J]) {
+    static_assert(J >= 1 && J <= 32 && (J & (J - 1)) == 0, "J must be a power of two <= 32");
+    begin_keys();
+    if constexpr (J % 4 == 0) {
+#pragma unroll
+        for (int k = 0; k < J; k += 4) {
+            uint32_t q[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) q[i] = __reduce_max_sync(kFull, amax_key(x[k + i]));
+            put_keys(k, q[0], q[1], q[2], q[3]);
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < J; ++k) put_key(k, __reduce_max_sync(kFull, amax_key(x[k])));
+    }
+    return publish_scales<T, J>();
+}
+
+template <typename T, bool VEC, int J, typename Emit>
+__device__ __forceinline__ void wire_blocks_raw(const T *src, const int (&valid)[J], Emit &&emit) {
+    Raw4<T> x[J];
+#pragma unroll
+    for (int j = 0; j < J; ++j) x[j] = load_raw4<T, VEC>(src + j * kBlock, valid[j]);
+    with_fast(scales_of_raw_blocks<T, J>(x), [&](auto fast) {
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            float v[4];
+            widen4(x[j], v);
+            wire4<decltype(fast)::value>(v, scale_of(j));
+            emit(j, v);
+        }
+    });
+}
+
+// The sender side alone: the codes of J consecutive blocks at src (as
+// wire_blocks_raw, loads raw until their block is quantised), handed to
+// emit(j, codes) as one word of 4 codes per lane; block j's scale is
+// scale_of(j).s.x afterwards.
+template <typename T, bool VEC, int J, typename Emit>
+__device__ __forceinline__ void quant_blocks_raw(const T *src, const int (&valid)[J], Emit &&emit) {
+    Raw4<T> x[J];
+#pragma unroll
+    for (int j = 0; j < J; ++j) x[j] = load_raw4<T, VEC>(src + j * kBlock, valid[j]);
+    with_fast(scales_of_raw_blocks<T, J>(x), [&](auto fast) {
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            float v[4];
+            widen4(x[j], v);
+            emit(j, quant4<decltype(fast)::value>(v, scale_of(j)));
+        }
+    });
+}
+
 // ------------------------------------------------------ 16-byte bf16 stores
 
 // Row pieces of 16 bytes for a bf16 block pair held as 4 values per lane per
@@ -252,11 +318,13 @@ __device__ __forceinline__ int vec_valid_in(size_t i0, size_t hi, Full) {
 #define RLX_JD 8
 #endif
 // 128-blocks per warp unit of the single-source FP8 kernels with bf16 data
-// (alltoall, all-gather).  8 blocks per alltoall unit halve the per-unit work
-// (indices, the scales' division) but measured slower in the library at the
-// prefill size (231 against 223 us), so both stay at 4.
+// (alltoall, all-gather).  The alltoall keeps its loads raw until each block
+// is converted (wire_blocks_raw), so 8 bf16 blocks fit the register budget of
+// 4 CTAs per SM (62 registers) and halve the per-unit work (indices, the
+// scales' division): 221.9 -> 173.6 us at the prefill size.  The all-gather
+// stores every block to all N rows and stays at 4.
 #ifndef RLX_J_A2A_BF16
-#define RLX_J_A2A_BF16 4
+#define RLX_J_A2A_BF16 8
 #endif
 #ifndef RLX_J_AG_BF16
 #define RLX_J_AG_BF16 4
