@@ -715,9 +715,10 @@ def workload_suite(dev, peak: float, reps: int = 20, scale: int = 1) -> dict:
 def quotient_ablation(dev, reps: int = 20) -> dict:
     """Profiling mode: what the correctly rounded quotient costs.  Times the
     FP8-wire operations with the product build (quotient fl32(x / s) by
-    Markstein corrections) and with two profiling builds of the same sources
-    (build.VARIANTS: x * fl32(448 / amax), and CUDA's IEEE division for every
-    element), on workload 4 (N=8 x fp32[16,777,216]) and on the bf16 prefill
+    Markstein corrections) and with the profiling builds of the same sources
+    (build.VARIANTS: x * fl32(448 / amax); CUDA's IEEE division for every
+    element; the codes from two bracketing products with the full quotient
+    only where they disagree), on workload 4 (N=8 x fp32[16,777,216]) and on the bf16 prefill
     buffers (N=8 x bf16[33,554,432]), inputs drawn on the device; and counts
     the quantised codes and DDA-tree results in which each variant differs
     from the product build."""
@@ -876,8 +877,8 @@ def main(argv=None):
                     help="profiling: divide the other workloads' counts by this")
     ap.add_argument("--quotient-ablation", action="store_true",
                     help="profiling: time the FP8 operations with the correctly rounded "
-                         "quotient against two profiling builds (reciprocal multiply, IEEE "
-                         "division for every element); --steps calls each")
+                         "quotient against three profiling builds (reciprocal multiply, IEEE "
+                         "division for every element, bracketing products); --steps calls each")
     ap.add_argument("--count", type=int, default=COUNT,
                     help="elements per rank (profiling cases only; the benchmark is 16,777,216)")
     ap.add_argument("--only", default="",

@@ -86,6 +86,9 @@ VARIANTS = {
     "recip_quotient": ["-DRLX_QUOTIENT=1"],
     # CUDA's IEEE division for every element
     "ieee_div_quotient": ["-DRLX_QUOTIENT=2"],
+    # the correctly rounded quotient's codes from two bracketing products,
+    # the full quotient only where the bracket is not decisive
+    "bracket_quotient": ["-DRLX_QUOTIENT=3"],
 }
 
 

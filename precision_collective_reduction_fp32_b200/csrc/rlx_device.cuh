@@ -249,12 +249,16 @@ __device__ __forceinline__ float warp_amax4(const float (&v)[4]) {
 // _build/, never the library the package loads):
 //   1  x * fl32(448 / amax), one multiply per element (the reciprocal form a
 //      faster quantiser would use; it changes some codes);
-//   2  __fdiv_rn(x, s) for every element (CUDA's IEEE division).
+//   2  __fdiv_rn(x, s) for every element (CUDA's IEEE division);
+//   3  the codes of the correctly rounded quotient from two bracketing
+//      products (see neg_codes4), with the full quotient only for blocks
+//      where the bracket is not decisive.  Gives the same codes as 0.
 #ifndef RLX_QUOTIENT
 #define RLX_QUOTIENT 0
 #endif
 constexpr int kQuotient = RLX_QUOTIENT;
-static_assert(kQuotient >= 0 && kQuotient <= 2, "RLX_QUOTIENT must be 0, 1 or 2");
+static_assert(kQuotient >= 0 && kQuotient <= 3, "RLX_QUOTIENT must be 0, 1, 2 or 3");
+constexpr bool kBracket = kQuotient == 3;
 
 // Scale of a block: s = fl32(amax / 448), and ny = -fl32(1 / s) when the fast
 // quotient may be used (s >= 2^-90), else 0.  (RLX_QUOTIENT=1: ny =
@@ -274,6 +278,8 @@ constexpr bool k2Term = RLX_QUOTIENT_2TERM && kQuotient == 0;
 
 // With the two-term reciprocal the scale also carries nlo = -y_lo, where
 // y_hi = RD(1/s) and y_lo = RN((1 - s*y_hi) * y) >= +0 (so nlo <= -0).
+// With RLX_QUOTIENT=3 (nhi, nlo) = (fl32(ny * (1 + 2^-21)),
+// fl32(ny * (1 - 2^-21))), the two bracketing multipliers.
 struct Scale {
     float s, ny, nhi, nlo;
 };
@@ -301,6 +307,10 @@ __device__ __forceinline__ Scale make_scale(float amax) {
     r.nhi = r.nlo = 0.0f;
     if constexpr (kQuotient == 0) {
         r = reciprocal_terms(r.s);
+    } else if constexpr (kBracket) {
+        r = reciprocal_terms(r.s);
+        r.nhi = __fmul_rn(r.ny, 1.0f + 0x1p-21f);
+        r.nlo = __fmul_rn(r.ny, 1.0f - 0x1p-21f);
     } else if constexpr (kQuotient == 1) {
         r.ny = r.s >= kMinFastScale ? -__fdiv_rn(kE4m3Max, amax) : 0.0f;
     } else {
@@ -324,7 +334,7 @@ __device__ __forceinline__ Scale2 pack(Scale sc) {
 constexpr int kWarpsPerCta = 8;
 struct alignas(16) WarpScratch {
     float4 scale[32];   // block k: (s, s, ny, ny)
-    float4 split[k2Term ? 32 : 1];   // block k: (nhi, nhi, nlo, nlo) (two-term reciprocal)
+    float4 split[k2Term || kBracket ? 32 : 1];   // block k: (nhi, nhi, nlo, nlo)
     uint32_t key[32];   // block k: its amax key
 };
 __device__ __forceinline__ WarpScratch &warp_scratch() {
@@ -362,7 +372,8 @@ __device__ __forceinline__ bool publish_scales() {
     const Scale own = make_scale(amax_of<T>(w.key[lane & (K - 1)]));
     if (lane < K) {
         w.scale[lane] = make_float4(own.s, own.s, own.ny, own.ny);
-        if constexpr (k2Term) w.split[lane] = make_float4(own.nhi, own.nhi, own.nlo, own.nlo);
+        if constexpr (k2Term || kBracket)
+            w.split[lane] = make_float4(own.nhi, own.nhi, own.nlo, own.nlo);
     }
     const bool fast = __all_sync(kFull, own.ny != 0.0f);
     __syncwarp();
@@ -383,7 +394,7 @@ __device__ __forceinline__ bool publish_scales(const uint32_t (&key)[K]) {
 }
 __device__ __forceinline__ Scale2 scale_of(int k) {
     const float4 v = warp_scratch().scale[k];
-    if constexpr (k2Term) {
+    if constexpr (k2Term || kBracket) {
         const float4 u = warp_scratch().split[k];
         return {f2(v.x, v.y), f2(v.z, v.w), f2(u.x, u.y), f2(u.z, u.w)};
     }
@@ -480,15 +491,43 @@ __device__ __forceinline__ void neg_quotients4(const float (&v)[4], const Scale2
     }
 }
 
+// The codes of -fl32(v/s) for 4 values of a block (byte k = element k).
+// RLX_QUOTIENT=3: E, the E4M3 encoding (round to nearest even, saturating),
+// is monotone, so if the codes of two values a and b agree, every value
+// between them has that code too.  With y = fl32(1/s) (relative error
+// <= 2^-24), the products a = fl32(v * fl32(-y * (1 + 2^-21))) and
+// b = fl32(v * fl32(-y * (1 - 2^-21))) lie, for every quotient in the fp32
+// normal range, at least 2^-21 - 4 * 2^-24 > 2^-24 (relative) beyond -v/s
+// on either side, while -fl32(v/s) lies within 2^-24 of it: the correctly
+// rounded quotient is bracketed.  (Quotients below the normal range have
+// code +-0, as do both products; v = +-0 gives -+0 everywhere.)  So where
+// E(a) == E(b) in every lane, E(a) is the code of the correctly rounded
+// quotient; a block where some lane's bracket straddles a rounding boundary
+// takes the full quotient.  Every lane of the warp calls this.
+template <bool Fast>
+__device__ __forceinline__ uint32_t neg_codes4(const float (&v)[4], const Scale2 &sc) {
+    if constexpr (kBracket) {
+        if (Fast || sc.ny.x != 0.0f) {
+            const float2 x0 = f2(v[0], v[1]), x1 = f2(v[2], v[3]);
+            const float2 a0 = __fmul2_rn(x0, sc.nhi), a1 = __fmul2_rn(x1, sc.nhi);
+            const float2 b0 = __fmul2_rn(x0, sc.nlo), b1 = __fmul2_rn(x1, sc.nlo);
+            const uint32_t ca = e4m3x2_from_f32(a0.x, a0.y) | (e4m3x2_from_f32(a1.x, a1.y) << 16);
+            const uint32_t cb = e4m3x2_from_f32(b0.x, b0.y) | (e4m3x2_from_f32(b1.x, b1.y) << 16);
+            if (__all_sync(kFull, ca == cb)) return ca;
+        }
+    }
+    float p[4];
+    neg_quotients4<Fast>(v, sc, p);
+    return e4m3x4_from_f32(p);
+}
+
 // Quantise 4 values of a block with scale sc: code = e4m3_rne_sat(fl32(v/s)).
 // The E4M3 encoding is symmetric in the sign (round to nearest even, the
 // saturation bound and zero included), so the codes of -q are the codes of q
 // with the sign bit of every byte flipped back.
 template <bool Fast = false>
 __device__ __forceinline__ uint32_t quant4(const float (&v)[4], const Scale2 &sc) {
-    float p[4];
-    neg_quotients4<Fast>(v, sc, p);
-    return e4m3x4_from_f32(p) ^ 0x80808080u;
+    return neg_codes4<Fast>(v, sc) ^ 0x80808080u;
 }
 
 // Dequantise 4 packed codes with scale s: fl32(e4m3(code) * s).  The
@@ -524,9 +563,19 @@ __device__ __forceinline__ void dequant4(uint32_t codes, float s, float (&y)[4])
 #endif
 template <bool Fast>
 __device__ __forceinline__ void wire4(float (&v)[4], const Scale2 &sc) {
+    const float ns = -sc.s.x;
+    if constexpr (kBracket) {
+        const uint32_t c = neg_codes4<Fast>(v, sc);
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const float2 w = e4m3x2_to_f32(k == 0 ? c & 0xffffu : c >> 16);
+            v[2 * k] = __fmul_rn(w.x, ns);
+            v[2 * k + 1] = __fmul_rn(w.y, ns);
+        }
+        return;
+    }
     float p[4];
     neg_quotients4<Fast>(v, sc, p);
-    const float ns = -sc.s.x;
 #if RLX_DEQ_FFMA2 && RLX_PACKED_F32X2
     const float nz = __fmul_rn(ns, 0.0f);   // -0: s >= 0
     const float2 ns2 = f2(ns, ns), nz2 = f2(nz, nz);
