@@ -22,7 +22,8 @@ from HBM.  `roofline` is the slowest single-kernel operation against the
 measured copy bandwidth, and `roofline.target` the FP8 DDA-tree allreduce
 (the fused low-precision allreduce the >= 16 MB target is quoted on).
 `e2e` is that one collective end to end: each step uploads the 512 MiB
-input from pinned host memory, runs it and downloads the 512 MiB result.
+input from pinned host memory, runs it and downloads the 512 MiB result, in
+column ranges so that the two PCIe directions overlap.
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference]
 
@@ -266,60 +267,101 @@ class Step:
         ]
 
 
+try:   # strided host<->device copies in one call (plumbing only)
+    from cuda.bindings import runtime as _rt
+except ImportError:
+    _rt = None
+
+
 class E2ETreeFp8:
     """End to end through the C ABI, one collective per step: copy the rank
     buffers from pinned host memory to the device, run the FP8 DDA-tree
     allreduce (fused dequantise-sum-requantise pass + all-gather pass) and
-    copy the result back to pinned host memory.  Uploads, kernels and
-    downloads run on three streams with two device batches, so step k's
-    upload and step k-1's download overlap step k's kernels.  Calling the
-    object with a step count returns the device time of those steps (ms),
-    from the first upload's start to the last download's end."""
+    copy the result back to pinned host memory.
 
-    def __init__(self, x_host: np.ndarray, dev):
+    Each step is cut into `slices` column ranges of the [N][count] rank rows
+    (multiples of the 128-element FP8 block, so every block and the result
+    are those of one call on the whole rows: the tree's result does not depend
+    on its chunking), and each range is uploaded, reduced by one
+    rlx_allreduce_tree call on the strided rows and downloaded on its own, on
+    three streams (uploads, kernels, downloads) with two device batches: the
+    upload of one range overlaps the download of an earlier one, so both
+    PCIe directions stay busy, and only one range's transfer is not
+    overlapped at the start and end.  Calling the object with a step count
+    returns the device time of those steps (ms), from the first upload's
+    start to the last download's end; `result(k)` is step k's host output
+    buffer."""
+
+    def __init__(self, x_host: np.ndarray, dev, slices: int = 8):
         import torch
         from precision_collective_reduction_fp32_b200 import binding as B
         self.B, self.torch = B, torch
         self.n, self.c = x_host.shape
-        self.wsb = B.rlx_workspace_bytes(B.RLX_COLL_ALLREDUCE_TREE, self.c, self.n, B.RLX_F32,
+        while slices > 1 and (self.c % slices or (self.c // slices) % BLOCK):
+            slices -= 1
+        self.slices, self.w = slices, self.c // slices
+        self.wsb = B.rlx_workspace_bytes(B.RLX_COLL_ALLREDUCE_TREE, self.w, self.n, B.RLX_F32,
                                          B.RLX_WIRE_FP8_E4M3)
         self.host_in = torch.from_numpy(x_host).pin_memory()
         self.host_out = [torch.empty((self.n, self.c), dtype=torch.float32).pin_memory()
                          for _ in range(2)]
         self.dx = [torch.empty((self.n, self.c), dtype=torch.float32, device=dev) for _ in range(2)]
         self.dy = [torch.empty_like(self.dx[0]) for _ in range(2)]
-        self.ws = [torch.empty(self.wsb, dtype=torch.uint8, device=dev) for _ in range(2)]
+        self.ws = torch.empty(max(self.wsb, 1), dtype=torch.uint8, device=dev)
         self.stream = torch.cuda.current_stream(dev)
         self.s_in, self.s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         self.h2d_bytes = self.d2h_bytes = self.n * self.c * 4
 
+    def result(self, k: int):
+        return self.host_out[k % 2]
+
+    def _copy_range(self, dst, src, lo: int, hi: int, h2d: bool, stream) -> None:
+        """Columns [lo, hi) of all N rows, src -> dst (both [N][count]): one
+        2-D copy (cudaMemcpy2DAsync) when cuda-python's runtime bindings are
+        importable, else one copy per row."""
+        if _rt is not None:
+            pitch, width = self.c * 4, (hi - lo) * 4
+            kind = (_rt.cudaMemcpyKind.cudaMemcpyHostToDevice if h2d
+                    else _rt.cudaMemcpyKind.cudaMemcpyDeviceToHost)
+            err, = _rt.cudaMemcpy2DAsync(dst[0, lo:].data_ptr(), pitch, src[0, lo:].data_ptr(), pitch,
+                                         width, self.n, kind, stream.cuda_stream)
+            if err != _rt.cudaError_t.cudaSuccess:
+                raise RuntimeError("cudaMemcpy2DAsync failed: %s" % err)
+            return
+        for r in range(self.n):
+            dst[r, lo:hi].copy_(src[r, lo:hi], non_blocking=True)
+
     def __call__(self, nsteps: int) -> float:
         torch, B = self.torch, self.B
-        n, c, sp = self.n, self.c, self.stream.cuda_stream or None
+        n, c, w, S = self.n, self.c, self.w, self.slices
+        sp = self.stream.cuda_stream or None
         ev = lambda: torch.cuda.Event(enable_timing=True)
         start = ev()
-        ev_in, ev_c, ev_out = ([ev() for _ in range(nsteps)] for _ in range(3))
+        ev_in, ev_c, ev_out = ([[ev() for _ in range(S)] for _ in range(nsteps)] for _ in range(3))
         start.record(self.s_in)
         for k in range(nsteps):
             b = k % 2
-            with torch.cuda.stream(self.s_in):
+            dx, dy, ho = self.dx[b], self.dy[b], self.host_out[b]
+            for i in range(S):
+                lo, hi = i * w, (i + 1) * w
+                with torch.cuda.stream(self.s_in):
+                    if k >= 2:
+                        self.s_in.wait_event(ev_c[k - 2][i])    # range i of batch b is free again
+                    self._copy_range(dx, self.host_in, lo, hi, True, self.s_in)
+                    ev_in[k][i].record(self.s_in)
+                self.stream.wait_event(ev_in[k][i])
                 if k >= 2:
-                    self.s_in.wait_event(ev_c[k - 2])      # batch b's input is free again
-                self.dx[b].copy_(self.host_in, non_blocking=True)
-                ev_in[k].record(self.s_in)
-            self.stream.wait_event(ev_in[k])
-            if k >= 2:
-                self.stream.wait_event(ev_out[k - 2])      # batch b's result was read out
-            B.rlx_allreduce_tree(self.dx[b].data_ptr(), self.dy[b].data_ptr(), c, c, n, B.RLX_F32,
-                                 B.RLX_WIRE_FP8_E4M3, B.RLX_SUM, self.ws[b].data_ptr(), self.wsb,
-                                 sp)
-            ev_c[k].record(self.stream)
-            with torch.cuda.stream(self.s_out):
-                self.s_out.wait_event(ev_c[k])
-                self.host_out[b].copy_(self.dy[b], non_blocking=True)
-                ev_out[k].record(self.s_out)
+                    self.stream.wait_event(ev_out[k - 2][i])    # its result was read out
+                B.rlx_allreduce_tree(dx[0, lo:].data_ptr(), dy[0, lo:].data_ptr(), w, c, n,
+                                     B.RLX_F32, B.RLX_WIRE_FP8_E4M3, B.RLX_SUM,
+                                     self.ws.data_ptr(), self.wsb, sp)   # raises on failure
+                ev_c[k][i].record(self.stream)
+                with torch.cuda.stream(self.s_out):
+                    self.s_out.wait_event(ev_c[k][i])
+                    self._copy_range(ho, dy, lo, hi, False, self.s_out)
+                    ev_out[k][i].record(self.s_out)
         torch.cuda.synchronize()
-        return start.elapsed_time(ev_out[-1])
+        return start.elapsed_time(ev_out[-1][-1])
 
 
 def run_gpu(args, rank: int, world: int) -> dict | None:
@@ -405,6 +447,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
     barrier()
     e2e_ms = max_over_ranks(e2e_run(Ke), dev)
     barrier()
+    e2e_slices = e2e_run.slices
     del e2e_run
     if rank != 0:
         return None
@@ -462,7 +505,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
                      "algorithmic_bytes": bytes_[dom], "peak_kind": peak_kind + " copy"},
         "gpu_launches": K * sum(KERNELS_PER_OP[n] for n in bytes_),
         "gpu_launches_breakdown_pass": K * sum(KERNELS_PER_OP[n] for n in bytes_),
-        "gpu_launches_e2e": Ke * KERNELS_PER_OP[TARGET_OP],
+        "gpu_launches_e2e": Ke * e2e_slices * KERNELS_PER_OP[TARGET_OP],
         "clocks": clk,
         "e2e": {"value": round(whole_job_gbs(world, e2e_bytes, Ke, e2e_ms), 1), "unit": "GB/s",
                 "h2d_bytes_per_step": NRANKS * count * 4, "d2h_bytes_per_step": NRANKS * count * 4,
@@ -470,7 +513,9 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
                 "operation": TARGET_OP,
                 "numerator": "the operation's algorithmic HBM bytes (%d per step)" % e2e_bytes,
                 "pcie_GBs": round(world * 2 * NRANKS * count * 4 * Ke / (e2e_ms * 1e-3) / 1e9, 1),
-                "overlap": "uploads, kernels and downloads on three streams, two device batches"},
+                "overlap": "each step in %d column ranges, each uploaded, reduced by one "
+                           "rlx_allreduce_tree call and downloaded; uploads, kernels and downloads "
+                           "on three streams, two device batches" % e2e_slices},
     }
     if TARGET_OP in per_op:
         t = per_op[TARGET_OP]
