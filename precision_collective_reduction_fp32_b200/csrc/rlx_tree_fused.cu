@@ -116,8 +116,18 @@ struct FusedArgs {
     TreePlan plan;
 };
 
-template <typename T, int NR, bool VEC, bool EXACT, bool FP8>
-__global__ void __launch_bounds__(kThreads, NR <= 8 ? 2 : 1)
+// CTAs per SM the kernel is compiled for (MINB, up to 8 ranks).  Both
+// passes' unit bodies share its registers: at 2 CTAs per SM they are not
+// spilled, at 4 the FP8 instantiations spill a little but twice the warps are
+// in flight.  The launcher takes the 2-per-SM form when the runs fit in one
+// wave of it (small messages, where the spills add latency: decode bf16 FP8
+// from a graph 10.9 against 11.8 us) and the 4-per-SM form beyond (prefill
+// bf16: native 205 -> 186 us, FP8 276 -> 244 us; fp32 FP8 at 8 x 16 Mi:
+// 229 -> 205 us).
+constexpr int kFusedMinbSmall = 2, kFusedMinbLarge = 4;
+
+template <typename T, int NR, bool VEC, bool EXACT, bool FP8, int MINB>
+__global__ void __launch_bounds__(kThreads, NR <= 8 ? MINB : 1)
 tree_fused_kernel(FusedArgs a) {
     __shared__ uint32_t s_ticket[2];
     __shared__ uint32_t s_done[RLX_MAX_RANKS];
@@ -270,14 +280,22 @@ cudaError_t launch_tree_fused(const void *send, void *recv, size_t count, size_t
     }
     return dispatch_fused(dtype, nranks, vec, [&]<typename T, int NR, bool VEC, bool EX>() {
         if (!make_tree_plan<T>(count, nranks, chunk, fp8, &a.plan)) return cudaErrorInvalidValue;
-        const void *k = !fp8 ? reinterpret_cast<const void *>(tree_fused_kernel<T, NR, VEC, EX, false>)
-                             : reinterpret_cast<const void *>(tree_fused_kernel<T, NR, VEC, EX, true>);
-        const int resident = resident_ctas(k);
-        if (resident <= 0) return cudaErrorInvalidValue;
         const size_t runs = static_cast<size_t>(a.plan.runs1) + a.plan.runs2;
-        const dim3 grid(static_cast<unsigned>(runs < static_cast<size_t>(resident) ? runs : resident));
-        if (!fp8) return launch_kernel(tree_fused_kernel<T, NR, VEC, EX, false>, grid, stream, a);
-        return launch_kernel(tree_fused_kernel<T, NR, VEC, EX, true>, grid, stream, a);
+        // the grid is at most one wave of resident CTAs of the form launched
+        auto go = [&]<int MINB>() -> cudaError_t {
+            auto *k = fp8 ? tree_fused_kernel<T, NR, VEC, EX, true, MINB>
+                          : tree_fused_kernel<T, NR, VEC, EX, false, MINB>;
+            const int resident = resident_ctas(reinterpret_cast<const void *>(k));
+            if (resident <= 0) return cudaErrorInvalidValue;
+            const dim3 grid(static_cast<unsigned>(runs < static_cast<size_t>(resident) ? runs : resident));
+            return launch_kernel(k, grid, stream, a);
+        };
+        const int small = resident_ctas(reinterpret_cast<const void *>(
+            fp8 ? tree_fused_kernel<T, NR, VEC, EX, true, kFusedMinbSmall>
+                : tree_fused_kernel<T, NR, VEC, EX, false, kFusedMinbSmall>));
+        if (small > 0 && runs <= static_cast<size_t>(small))
+            return go.template operator()<kFusedMinbSmall>();
+        return go.template operator()<kFusedMinbLarge>();
     });
 }
 
