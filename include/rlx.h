@@ -142,6 +142,11 @@ RLX_API rlx_status rlx_allreduce_flat(const void *send, void *recv, size_t count
  *   FP8 wire: pass 1 reduces the dequantised FP8 contributions and quantises
  *     the reduced chunk again (second quantisation) into `workspace`; pass 2
  *     dequantises it into every rank.
+ * Small messages (up to a few waves of the GPU) run both passes in one kernel
+ * launch over thread-block clusters: each cluster reduces a contiguous range
+ * of the chunks, synchronises its CTAs with the cluster barrier and gathers
+ * the same range; larger ones run the passes as two launches.  The results
+ * are the same bytes either way.
  * workspace: device memory of at least rlx_workspace_bytes(RLX_COLL_ALLREDUCE_TREE,
  * ...) bytes, 16-byte aligned, not overlapping send/recv; may be NULL when that
  * size is 0.  Its contents on return are unspecified.  Same-stream calls may

@@ -250,6 +250,10 @@ rlx_status rlx_allreduce_tree(const void *send, void *recv, size_t count, size_t
         ws_scales = reinterpret_cast<float *>(ws_codes + nblk * RLX_BLOCK);
     }
     const bool vec = vec_ok(wire, es, {send, recv}, {stride});
+    // small messages: both passes in one launch over thread-block clusters
+    if (rlx::tree_cluster_wanted(count, nranks, chunk, dtype, wire))
+        return from_cuda(rlx::launch_tree_cluster(send, recv, count, stride, nranks, chunk, dtype,
+                                                  wire, ws_codes, ws_scales, vec, s));
     cudaError_t e = rlx::launch_tree_reduce(send, recv, count, stride, nranks, chunk, dtype, wire,
                                             ws_codes, ws_scales, vec, s);
     if (e != cudaSuccess) return from_cuda(e);

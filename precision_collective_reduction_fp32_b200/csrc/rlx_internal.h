@@ -64,6 +64,15 @@ cudaError_t launch_tree_gather(void *recv, size_t count, size_t stride, int nran
                                const uint8_t *ws_codes, const float *ws_scales, bool vec,
                                cudaStream_t stream);
 
+// DDA-tree in one launch over thread-block clusters (rlx_tree_cluster.cu):
+// the same arguments and results as the two passes above.  tree_cluster_wanted
+// says whether a call is small enough for it to be the faster path.
+bool tree_cluster_wanted(size_t count, int nranks, size_t chunk, rlx_dtype dtype, rlx_wire wire);
+cudaError_t launch_tree_cluster(const void *send, void *recv, size_t count, size_t stride,
+                                int nranks, size_t chunk, rlx_dtype dtype, rlx_wire wire,
+                                uint8_t *ws_codes, float *ws_scales, bool vec,
+                                cudaStream_t stream);
+
 // DDA-tree in one launch with chunk-ready counts (rlx_tree_fused.cu).
 // workspace: RLX_TREE_SYNC_BYTES of sync words (zero on entry), then on the
 // FP8 wire the payload.  status may be null.

@@ -495,10 +495,12 @@ __device__ __forceinline__ void tree_reduce_fp8_unit(uint32_t u, const T *send, 
 
 // Pass 2, native: unit g = (chunk c, kWarpVecs vectors of it); chunk c of
 // row c -> chunk c of every other row.
+// (Rows r0, r0 + rstep, ... only: a unit's rows can be split among warps.)
 template <typename T, bool VEC>
 __device__ __forceinline__ void tree_gather_native_unit(uint32_t g, T *recv, size_t count,
                                                         size_t stride, int n, size_t chunk,
-                                                        const FastDiv &per_chunk) {
+                                                        const FastDiv &per_chunk, int r0 = 0,
+                                                        int rstep = 1) {
     const uint32_t c = fast_div(g, per_chunk);
     const size_t lo = static_cast<size_t>(c) * chunk;
     if (lo >= count) return;
@@ -509,18 +511,20 @@ __device__ __forceinline__ void tree_gather_native_unit(uint32_t g, T *recv, siz
         int valid[kUnroll];
         // the owner's chunk was just written by pass 1: read it through L2
         load_unit<T, VEC, true>(recv + c * stride + lo, unit, len, full, a, valid);
-        for (int r = 0; r < n; ++r)
+        for (int r = r0; r < n; r += rstep)
             if (static_cast<uint32_t>(r) != c)
                 store_unit<T, VEC>(recv + r * stride + lo, unit, a, valid);
     });
 }
 
-// Pass 2, FP8: unit g = kJd payload blocks, dequantised into every row.
+// Pass 2, FP8: unit g = kJd payload blocks, dequantised into every row
+// (rows r0, r0 + rstep, ... only: a unit's rows can be split among warps).
 template <typename T, bool VEC>
 __device__ __forceinline__ void tree_gather_fp8_unit(uint32_t g, T *recv, size_t count,
                                                      size_t stride, int n,
                                                      const uint8_t *ws_codes,
-                                                     const float *ws_scales) {
+                                                     const float *ws_scales, int r0 = 0,
+                                                     int rstep = 1) {
     const size_t nblk = (count + kBlock - 1) / kBlock;
     const int e0 = lane_id() * 4;
     const size_t b0 = static_cast<size_t>(g) * kJd;
@@ -542,7 +546,7 @@ __device__ __forceinline__ void tree_gather_fp8_unit(uint32_t g, T *recv, size_t
                 q[p] = make_uint4(bf16x2_bits(y[0][0], y[0][1]), bf16x2_bits(y[0][2], y[0][3]),
                                   bf16x2_bits(y[1][0], y[1][1]), bf16x2_bits(y[1][2], y[1][3]));
             }
-            for (int r = 0; r < n; ++r) {
+            for (int r = r0; r < n; r += rstep) {
                 T *dst = recv + r * stride + b0 * kBlock + 8 * l;
 #pragma unroll
                 for (int p = 0; p < kJd / 2; ++p)
@@ -565,7 +569,7 @@ __device__ __forceinline__ void tree_gather_fp8_unit(uint32_t g, T *recv, size_t
                 dequant4(codes, __ldcg(ws_scales + b), y[j]);
             }
         }
-        for (int r = 0; r < n; ++r) {
+        for (int r = r0; r < n; r += rstep) {
             T *dst = recv + r * stride + b0 * kBlock + e0;
 #pragma unroll
             for (int j = 0; j < kJd; ++j) store4<T, VEC>(dst + j * kBlock, valid[j], y[j]);

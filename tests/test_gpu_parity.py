@@ -214,6 +214,18 @@ def test_tree_in_place_mid_size(wire, count, inplace):
     assert _bits_equal(got, oracle.allreduce_tree(x, wire=ORC_WIRE[wire]))
 
 
+@pytest.mark.parametrize("wire", WIRES)
+@pytest.mark.parametrize("dtype,count", [(None, 4_194_304 + 77), ("bf16", 8_388_608 + 2 * 128 + 77)])
+@pytest.mark.parametrize("inplace", [False, True])
+def test_tree_two_launch_ragged(wire, dtype, count, inplace):
+    """Counts past the range of the one-launch cluster path, so the DDA-tree
+    runs as its two launches, with a partial last block, in place and not
+    (the parity cases above are small enough for the cluster path)."""
+    x = synth.rank_buffers(4, count=count, nranks=8, dtype=dtype)
+    got = _run_allreduce("tree", x, count, count, wire, inplace=inplace)
+    assert _bits_equal(got, oracle.allreduce_tree(x, wire=ORC_WIRE[wire]))
+
+
 @pytest.mark.parametrize("algo", ["flat", "tree"])
 def test_bf16_fp8_large_ragged(algo):
     """bf16 on the FP8 wire past the small-message threshold (>= 32768 blocks,
