@@ -42,11 +42,11 @@ struct ClusterArgs {
     size_t count, stride, chunk;
     uint8_t *ws_codes;
     float *ws_scales;
-    uint32_t groups;   // all-gather units = groups
-    uint32_t units1;   // FP8: reduce-scatter units (native: per1 per chunk)
-    uint32_t per_group;   // reduce-scatter units per group
-    uint32_t groups_per_cluster;
-    FastDiv per1, per2;   // native: units per chunk of the two passes
+    uint32_t groups;               // groups = all-gather units
+    uint32_t units1;               // FP8: reduce-scatter units (unused on the native wire)
+    uint32_t per_group;            // reduce-scatter units (and warps) per group
+    uint32_t groups_per_cluster;   // kClusterWarps / per_group
+    FastDiv per1, per2;            // native: units per chunk of the two passes
     int n;
 };
 
