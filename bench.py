@@ -135,9 +135,9 @@ def source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(op: str):
+def recorded_traffic(op: str, count: int = COUNT):
     """dram bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel sources (else None)."""
+    on the current kernel sources and at this count per rank (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
@@ -145,7 +145,7 @@ def recorded_traffic(op: str):
     except (OSError, ValueError):
         return None
     e = rec.get(op)
-    if not e or e.get("src_sha") != source_hash():
+    if not e or e.get("src_sha") != source_hash() or e.get("count") != count:
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -466,7 +466,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
     single = [n for n in per_op_ms if KERNELS_PER_OP[n] == 1]
     dom = max(single, key=lambda n: per_op_ms[n])
     dom_gbs = per_op[dom]["GB/s"]
-    traffic = recorded_traffic(dom)
+    traffic = recorded_traffic(dom, count)
     peak_desc = ("%s HBM copy bandwidth (read + write bytes of a 1 GiB device copy); read-heavy "
                  "operations can exceed it, so every fraction is also given against the nominal "
                  "%.0f GB/s" % (peak_kind, HBM_NOMINAL_GBS))
@@ -524,7 +524,7 @@ def run_gpu(args, rank: int, world: int) -> dict | None:
             "workload": "N=8 x fp32[16,777,216] (64 MiB per rank)",
             "us": t["us"], "achieved": t["GB/s"], "peak": peak, "unit": "GB/s",
             "frac": t["frac"], "frac_nominal": t["frac_nominal"],
-            "algorithmic_bytes": bytes_[TARGET_OP], "traffic": recorded_traffic(TARGET_OP),
+            "algorithmic_bytes": bytes_[TARGET_OP], "traffic": recorded_traffic(TARGET_OP, count),
             "goal": ">= 0.70 of the HBM roofline for the fused FP8 allreduce on >= 16 MB messages"}
     if world == 1 and not args.only and not args.no_latency:
         res["small_messages"] = small_message_latency(dev)

@@ -64,6 +64,8 @@ def test_recorded_traffic_needs_matching_kernels(monkeypatch):
     if rec is None:
         pytest.skip("no traffic record for the current kernel sources")
     assert 0.9 * 1024 * MIB < rec <= 1024 * MIB
+    # a record taken at another size does not describe this launch
+    assert bench.recorded_traffic("allreduce_flat_fp8", bench.COUNT // 4) is None
     monkeypatch.setattr(bench, "source_hash", lambda: real[::-1])
     assert bench.recorded_traffic("allreduce_flat_fp8") is None
 
