@@ -28,8 +28,10 @@ namespace {
 
 namespace cg = cooperative_groups;
 
+// CTAs per cluster (measured from a CUDA graph, decode bf16 tree native /
+// FP8: 2 CTAs 3.2 / 4.9 us, 4 CTAs 3.4 / 5.3 us, 8 CTAs 3.7 / 5.9 us).
 #ifndef RLX_TREE_CLUSTER_CTAS
-#define RLX_TREE_CLUSTER_CTAS 4
+#define RLX_TREE_CLUSTER_CTAS 2
 #endif
 constexpr uint32_t kClusterCtas = RLX_TREE_CLUSTER_CTAS;
 constexpr uint32_t kClusterWarps = kClusterCtas * kWarpsPerCta;
@@ -139,8 +141,8 @@ cudaLaunchConfig_t cluster_config(dim3 grid, cudaStream_t stream, cudaLaunchAttr
 
 // Whether a call takes the cluster path: while its clusters fill at most a
 // few waves of the GPU (2 CTAs per SM).  Measured against the two launches
-// (from a CUDA graph, N = 8): decode bf16 [32, 8192] native 3.4 against
-// 4.5 us, FP8 5.3 against 7.4 us; quick-start fp32 [10, 20] FP8 3.7 against
+// (from a CUDA graph, N = 8): decode bf16 [32, 8192] native 3.2 against
+// 4.5 us, FP8 4.9 against 7.4 us; quick-start fp32 [10, 20] FP8 3.4 against
 // 6.6 us; at 3.5 waves (2 Mi bf16 / 1 Mi fp32 per rank) native and fp32 FP8
 // still gain ~1 us, bf16 FP8 loses 1.5 us (its issue-bound reduce-scatter
 // runs at 4 CTAs per SM in its own kernel); from 4 Mi fp32 / 8 Mi bf16 per
@@ -165,7 +167,7 @@ bool tree_cluster_wanted(size_t count, int nranks, size_t chunk, rlx_dtype dtype
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return false;
-    const size_t wave = static_cast<size_t>(sms) * 2 / kClusterCtas;
+    const size_t wave = static_cast<size_t>(sms) * 2 / kClusterCtas;   // clusters per wave
     return clusters <= wave * (fp8 && bf16 ? 1 : 4);
 }
 
