@@ -89,11 +89,11 @@ flat_native_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
     });
 }
 
-// DDA-flat, FP8: unit u = the kBpu<T> blocks from block u*kBpu<T> on.
-template <typename T, int NR, bool VEC, bool EXACT>
+// DDA-flat, FP8: unit u = the BPU blocks from block u*BPU on (BPU = kBpu<T>,
+// or 1 for small bf16 messages, see launch_allreduce_flat).
+template <typename T, int NR, bool VEC, bool EXACT, int BPU>
 __global__ void __launch_bounds__(kThreads, kMinBlocksFp8Flat<NR>)
 flat_fp8_kernel(const T *send, T *recv, size_t count, size_t stride, int n) {
-    constexpr int BPU = kBpu<T>;
     const uint32_t units = static_cast<uint32_t>((count + BPU * kBlock - 1) / (BPU * kBlock));
     const bool wide = rows_16b(recv, stride);
     with_rank_count<NR, EXACT>(n, [&](auto nn) {
@@ -225,6 +225,17 @@ cudaError_t launch(K kernel, size_t units, size_t units_per_cta, cudaStream_t st
 
 constexpr size_t kWarps = kThreads / 32;
 
+// Below one wave of warps (148 SMs x 32), a flat FP8 call on bf16 is bound by
+// the latency of each warp's unit, not by bandwidth: units of one block
+// instead of two halve that chain and double the warps working on it
+// (decode bf16 8 x [32, 8192] from a CUDA graph: 2.7 against 3.2 us).  The
+// cluster-form tree keeps two-block units: with one-block units it measured
+// slower (5.4 against 5.0 us at the same size).
+#ifndef RLX_SMALL_BPU1
+#define RLX_SMALL_BPU1 1
+#endif
+constexpr size_t kSmallUnits = 148 * 32;
+
 }  // namespace
 
 cudaError_t launch_allreduce_flat(const void *send, void *recv, size_t count, size_t stride,
@@ -241,8 +252,11 @@ cudaError_t launch_allreduce_flat(const void *send, void *recv, size_t count, si
                           count, stride, nranks);
         }
         const size_t units = (count + kBpu<T> * kBlock - 1) / (kBpu<T> * kBlock);
-        return launch(flat_fp8_kernel<T, NR, VEC, EX>, units, kWarps * kPfFlat, stream, s, r, count,
-                      stride, nranks);
+        if (kBpu<T> > 1 && RLX_SMALL_BPU1 && units < kSmallUnits)
+            return launch(flat_fp8_kernel<T, NR, VEC, EX, 1>, units * kBpu<T>, kWarps * kPfFlat,
+                          stream, s, r, count, stride, nranks);
+        return launch(flat_fp8_kernel<T, NR, VEC, EX, kBpu<T>>, units, kWarps * kPfFlat, stream, s,
+                      r, count, stride, nranks);
     });
 }
 
