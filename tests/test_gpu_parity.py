@@ -156,7 +156,7 @@ def test_e4m3_hardware_conversion_below_band():
 # ------------------------------------------------------------------ allreduce
 
 AR_CASES = [(n, c) for n in (2, 3, 8) for c in (1, 7, 127, 128, 129, 1000, 3 * 128 * 8 + 5)] + \
-           [(4, 4096), (5, 1003), (16, 2000), (8, 65536 + 4), (8, 128 * 1024 + 3)]
+           [(4, 4096), (5, 1003), (16, 2000), (12, 3005), (8, 65536 + 4), (8, 128 * 1024 + 3)]
 
 
 def _run_allreduce(algo, x, count, stride, wire, inplace=False, offset=0):
